@@ -1,0 +1,327 @@
+"""Pins for the float64 oracle: results fixed by mathematics or by library routines.
+
+Each test ties the oracle to something other than itself: torch SDPA and
+autograd, central finite differences, closed forms derived by hand, brute-force
+rank counting, and invariants of the softmax. The mutation tests at the end
+plant plausible mistakes in copies of the oracle and check that a pin fails.
+"""
+import inspect
+import math
+import types
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import gated_attention as ga
+from tests.oracle_refs import rel_err, sdpa_dense_causal, sdpa_gated
+
+TOL = 1e-10
+
+
+def _rand(seed, B, Hq, Hkv, N, d, block, s_std=math.sqrt(2.0), qkv_std=1.0):
+    rng = np.random.default_rng(seed)
+    Nb = -(-N // block)
+    Q = rng.standard_normal((B, Hq, N, d)) * qkv_std
+    K = rng.standard_normal((B, Hkv, N, d)) * qkv_std
+    V = rng.standard_normal((B, Hkv, N, d))
+    S = rng.standard_normal((B, Hq, Nb, Nb)) * s_std
+    dO = rng.standard_normal((B, Hq, N, d))
+    return Q, K, V, S, dO
+
+
+# ---------------------------------------------------------------- textbook cases
+
+@pytest.mark.parametrize("shape", [(1, 2, 2, 64, 16, 16), (2, 4, 2, 48, 8, 8), (1, 2, 1, 40, 8, 16)])
+def test_gates_one_is_dense_causal(shape):
+    """Gates forced to 1 with every block kept reduces to dense causal attention."""
+    B, Hq, Hkv, N, d, bs = shape
+    Q, K, V, S, _ = _rand(1, B, Hq, Hkv, N, d, bs)
+    O, LSE = oracle.gated_attention_forward(Q, K, V, S, bs, gate="ones")
+    O_ref, LSE_ref = sdpa_dense_causal(Q, K, V)
+    assert rel_err(O, O_ref) < TOL
+    assert rel_err(LSE, LSE_ref) < TOL
+
+
+def test_single_block_is_dense_causal():
+    """block = N: there is no history, so the method is plain causal attention."""
+    Q, K, V, _, dO = _rand(2, 1, 2, 2, 32, 8, 32)
+    S = np.random.default_rng(3).standard_normal((1, 2, 1, 1))
+    O, LSE = oracle.gated_attention_forward(Q, K, V, S, 32)
+    O_ref, LSE_ref = sdpa_dense_causal(Q, K, V)
+    assert rel_err(O, O_ref) < TOL and rel_err(LSE, LSE_ref) < TOL
+    *_, dS, _ = oracle.gated_attention_backward(Q, K, V, S, dO, 32)
+    assert np.all(dS == 0.0)
+
+
+def test_closed_form_three_tokens():
+    """Hand-derived case, block = 1 (per-token units), d = 1, q = 0.
+
+    Row 2 has history {0, 1} with scores (ln 3, 0): gates (3/4, 1/4); the
+    current token has bias 0; all q.k are 0. Softmax weights are therefore
+    (3/8, 1/8, 1/2); with v = (1, 2, 3) the output is 17/8 and LSE = ln 2.
+    With dO = 1 on row 2: dZ = P (v - O) = (-27/64, -1/64, 28/64), so
+    G = (-27/64, -1/64) and dS = G - g * sum(G) = (-3/32, +3/32).
+    Row 1 has a single historical token: gate 1, weights (1/2, 1/2).
+    """
+    Q = np.zeros((1, 1, 3, 1))
+    K = np.array([1.0, -2.0, 0.5]).reshape(1, 1, 3, 1)
+    V = np.array([1.0, 2.0, 3.0]).reshape(1, 1, 3, 1)
+    S = np.zeros((1, 1, 3, 3))
+    S[0, 0, 2, 0] = math.log(3.0)
+    S[0, 0, 1, 0] = 5.0
+    O, LSE = oracle.gated_attention_forward(Q, K, V, S, 1)
+    assert np.allclose(O[0, 0, :, 0], [1.0, 1.5, 17.0 / 8.0], rtol=0, atol=1e-14)
+    assert np.allclose(LSE[0, 0], [0.0, math.log(2.0), math.log(2.0)], rtol=0, atol=1e-14)
+    dO = np.zeros((1, 1, 3, 1))
+    dO[0, 0, 2, 0] = 1.0
+    dQ, dK, dV, dS, Gs = oracle.gated_attention_backward(Q, K, V, S, dO, 1)
+    assert np.allclose(Gs[0, 0, 2, :2], [-27 / 64, -1 / 64], atol=1e-14)
+    assert np.allclose(dS[0, 0, 2, :2], [-3 / 32, 3 / 32], atol=1e-14)
+    assert np.allclose(dV[0, 0, :, 0], [3 / 8, 1 / 8, 1 / 2], atol=1e-14)
+
+
+def test_constant_scores_give_uniform_gates():
+    """A constant score row gives g = 1/|A|, i.e. log-gate -ln r (train) or -ln K."""
+    S = np.full((1, 1, 9, 9), 0.7)
+    idx, cnt, logg, _ = oracle.select_blocks(S, 9, None, mode=oracle.TRAIN)
+    for r in range(1, 9):
+        assert np.allclose(logg[0, 0, r, :r], -math.log(r), atol=1e-15)
+    idx, cnt, logg, _ = oracle.select_blocks(S, 9, 3, mode=oracle.SPARSE)
+    for r in range(4, 9):
+        assert cnt[0, 0, r] == 3
+        assert list(idx[0, 0, r, :3]) == [0, 1, 2]  # ties resolve to the lowest indices
+        assert np.allclose(logg[0, 0, r, :3], -math.log(3), atol=1e-15)
+
+
+# ------------------------------------------------------------ library cross-check
+
+CASES = [
+    # B, Hq, Hkv, N, d, block
+    (1, 2, 2, 64, 16, 16),
+    (1, 4, 2, 96, 8, 16),
+    (2, 2, 1, 40, 8, 16),    # ragged last block
+    (1, 2, 2, 24, 4, 1),     # per-token context units
+]
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_train_matches_sdpa_autograd(case):
+    B, Hq, Hkv, N, d, bs = case
+    Q, K, V, S, dO = _rand(10 + N, B, Hq, Hkv, N, d, bs)
+    O, LSE = oracle.gated_attention_forward(Q, K, V, S, bs)
+    dQ, dK, dV, dS, _ = oracle.gated_attention_backward(Q, K, V, S, dO, bs)
+    ref = sdpa_gated(Q, K, V, S, bs, dO=dO)
+    for name, x in dict(O=O, LSE=LSE, dQ=dQ, dK=dK, dV=dV, dS=dS).items():
+        assert rel_err(x, ref[name]) < 1e-9, name
+
+
+@pytest.mark.parametrize("renormalise", [True, False])
+@pytest.mark.parametrize("topk", [0, 1, 3])
+def test_sparse_matches_sdpa_autograd(topk, renormalise):
+    B, Hq, Hkv, N, d, bs = 1, 4, 2, 128, 8, 16
+    Q, K, V, S, dO = _rand(20 + topk, B, Hq, Hkv, N, d, bs)
+    kw = dict(mode=oracle.SPARSE, topk=topk, renormalise=renormalise)
+    O, LSE = oracle.gated_attention_forward(Q, K, V, S, bs, **kw)
+    dQ, dK, dV, dS, _ = oracle.gated_attention_backward(Q, K, V, S, dO, bs, **kw)
+    ref = sdpa_gated(Q, K, V, S, bs, mode="sparse", topk=topk, renormalise=renormalise, dO=dO)
+    for name, x in dict(O=O, LSE=LSE, dQ=dQ, dK=dK, dV=dV, dS=dS).items():
+        assert rel_err(x, ref[name]) < 1e-9, name
+
+
+# ---------------------------------------------------------- finite differences
+
+def _fd_check(Q, K, V, S, bs, W, n_pick=24, seed=0, eps=1e-6, bwd=None):
+    bwd = bwd or oracle.gated_attention_backward
+    rng = np.random.default_rng(seed)
+
+    def loss(Q_, K_, V_, S_):
+        O, _ = oracle.gated_attention_forward(Q_, K_, V_, S_, bs)
+        return float(np.sum(W * O))
+
+    dQ, dK, dV, dS, _ = bwd(Q, K, V, S, W, bs)
+    worst = 0.0
+    for name, X, dX in (("Q", Q, dQ), ("K", K, dK), ("V", V, dV), ("S", S, dS)):
+        flat = np.flatnonzero(np.ones(X.shape, dtype=bool))
+        if name == "S":  # only historical entries (c < r) feed the method
+            r = np.arange(X.shape[2])[:, None]
+            c = np.arange(X.shape[3])[None, :]
+            flat = np.flatnonzero(np.broadcast_to(c < r, X.shape))
+        pick = rng.choice(flat, size=min(n_pick, flat.size), replace=False)
+        for f in pick:
+            ix = np.unravel_index(f, X.shape)
+            args = {"Q": Q, "K": K, "V": V, "S": S}
+            Xp = X.copy(); Xp[ix] += eps
+            Xm = X.copy(); Xm[ix] -= eps
+            args[name] = Xp; lp = loss(**{k + "_": v for k, v in args.items()})
+            args[name] = Xm; lm = loss(**{k + "_": v for k, v in args.items()})
+            num = (lp - lm) / (2 * eps)
+            worst = max(worst, abs(num - dX[ix]) / max(1.0, abs(num)))
+    return worst
+
+
+def test_finite_differences_tiny():
+    """dQ, dK, dV and dS agree with central differences (N=32, d=8, block=4)."""
+    Q, K, V, S, W = _rand(5, 1, 2, 1, 32, 8, 4)
+    assert _fd_check(Q, K, V, S, 4, W) < 1e-6
+
+
+# -------------------------------------------------------------------- invariants
+
+def test_gate_rows_sum_to_one():
+    S = np.random.default_rng(7).standard_normal((2, 3, 12, 12)) * math.sqrt(2)
+    for mode, k in ((oracle.TRAIN, None), (oracle.SPARSE, 4)):
+        idx, cnt, logg, _ = oracle.select_blocks(S, 12, k, mode=mode)
+        for b in range(2):
+            for h in range(3):
+                for r in range(1, 12):
+                    n = cnt[b, h, r]
+                    assert abs(np.exp(logg[b, h, r, :n]).sum() - 1.0) < 1e-14
+
+
+def test_dS_rows_sum_to_zero_and_G_rows_cancel():
+    Q, K, V, S, dO = _rand(8, 1, 2, 2, 80, 8, 16)
+    for kw in ({}, dict(mode=oracle.SPARSE, topk=2)):
+        *_, dS, Gs = oracle.gated_attention_backward(Q, K, V, S, dO, 16, **kw)
+        assert np.max(np.abs(dS.sum(-1))) < 1e-12
+        # rows of dZ sum to zero, so block sums over a query block cancel
+        assert np.max(np.abs(np.nansum(Gs, -1))) < 1e-12
+
+
+def test_score_row_shift_invariance():
+    Q, K, V, S, dO = _rand(9, 1, 2, 2, 64, 8, 16)
+    shift = np.random.default_rng(1).standard_normal((1, 2, 4, 1)) * 5
+    for kw in ({}, dict(mode=oracle.SPARSE, topk=2)):
+        O1, L1 = oracle.gated_attention_forward(Q, K, V, S, 16, **kw)
+        O2, L2 = oracle.gated_attention_forward(Q, K, V, S + shift, 16, **kw)
+        assert rel_err(O2, O1) < 1e-12 and rel_err(L2, L1) < 1e-12
+        dS1 = oracle.gated_attention_backward(Q, K, V, S, dO, 16, **kw)[3]
+        dS2 = oracle.gated_attention_backward(Q, K, V, S + shift, dO, 16, **kw)[3]
+        assert rel_err(dS2, dS1) < 1e-9
+
+
+def test_full_budget_topk_equals_training():
+    Q, K, V, S, dO = _rand(11, 1, 2, 1, 96, 8, 16)
+    O1, L1 = oracle.gated_attention_forward(Q, K, V, S, 16)
+    for k in (5, 6, 100):
+        O2, L2 = oracle.gated_attention_forward(Q, K, V, S, 16, mode=oracle.SPARSE, topk=k)
+        assert np.array_equal(O1, O2) and np.array_equal(L1, L2)
+
+
+def test_gqa_equals_repeated_kv_heads():
+    Q, K, V, S, dO = _rand(12, 1, 4, 2, 48, 8, 16)
+    Kr, Vr = np.repeat(K, 2, axis=1), np.repeat(V, 2, axis=1)
+    O1, L1 = oracle.gated_attention_forward(Q, K, V, S, 16)
+    O2, L2 = oracle.gated_attention_forward(Q, Kr, Vr, S, 16)
+    assert rel_err(O1, O2) < 1e-14 and rel_err(L1, L2) < 1e-14
+    g1 = oracle.gated_attention_backward(Q, K, V, S, dO, 16)
+    g2 = oracle.gated_attention_backward(Q, Kr, Vr, S, dO, 16)
+    assert rel_err(g1[0], g2[0]) < 1e-13
+    assert rel_err(g1[1], g2[1].reshape(1, 2, 2, 48, 8).sum(2)) < 1e-13
+    assert rel_err(g1[2], g2[2].reshape(1, 2, 2, 48, 8).sum(2)) < 1e-13
+    assert rel_err(g1[3], g2[3]) < 1e-13
+
+
+def test_naive_equals_blockwise():
+    Q, K, V, S, _ = _rand(13, 1, 2, 1, 48, 8, 8)
+    for kw in ({}, dict(mode=oracle.SPARSE, topk=2), dict(mode=oracle.SPARSE, topk=2, renormalise=False)):
+        O1, L1 = oracle.gated_attention_forward(Q, K, V, S, 8, **kw)
+        O2, L2, _ = oracle.gated_attention_naive(Q, K, V, S, 8, **kw)
+        assert rel_err(O1, O2) < 1e-13 and rel_err(L1, L2) < 1e-13
+
+
+# ------------------------------------------------------------------------ Top-K
+
+def _brute_topk(s, r, k):
+    """Selected set by rank counting: c is kept iff fewer than k blocks beat it."""
+    keep = []
+    for c in range(r):
+        beats = sum(1 for c2 in range(r) if s[c2] > s[c] or (s[c2] == s[c] and c2 < c))
+        if beats < k:
+            keep.append(c)
+    return keep
+
+
+def test_topk_against_brute_force_with_ties():
+    rng = np.random.default_rng(14)
+    for trial in range(40):
+        r = int(rng.integers(0, 40))
+        s = rng.integers(-2, 3, size=r).astype(np.float64)
+        s[rng.random(r) < 0.2] = -0.0
+        for k in (0, 1, 3, 8, 50):
+            got = list(oracle.attended_blocks(s, r, oracle.SPARSE, k))
+            assert got == _brute_topk(s, r, k), (trial, k)
+
+
+def test_negative_zero_equals_positive_zero():
+    s = np.array([0.0, -0.0, 0.0, -0.0, -1.0])
+    assert list(oracle.attended_blocks(s, 5, oracle.SPARSE, 2)) == [0, 1]
+    s2 = np.array([-0.0, 0.0, -0.0])
+    assert list(oracle.attended_blocks(s2, 3, oracle.SPARSE, 1)) == [0]
+
+
+# ----------------------------------------------------------------------- decode
+
+@pytest.mark.parametrize("L", [64, 80, 127])
+def test_decode_equals_last_prefill_row(L):
+    """Decode at position L-1 equals row L-1 of sparse prefill with the same score row."""
+    rng = np.random.default_rng(L)
+    B, Hq, Hkv, d, bs, k = 2, 4, 2, 8, 8, 3
+    Nb = -(-L // bs)
+    Q = rng.standard_normal((B, Hq, L, d))
+    K = rng.standard_normal((B, Hkv, L, d))
+    V = rng.standard_normal((B, Hkv, L, d))
+    S_dec = rng.standard_normal((B, Hq, Nb)) * math.sqrt(2)
+    S = rng.standard_normal((B, Hq, Nb, Nb))
+    S[:, :, Nb - 1, :] = S_dec
+    O, LSE = oracle.gated_attention_forward(Q, K, V, S, bs, mode=oracle.SPARSE, topk=k)
+    Od, Ld = oracle.gated_decode(Q[:, :, L - 1], K, V, S_dec, L, bs, k)
+    assert rel_err(Od, O[:, :, L - 1]) < 1e-13 and rel_err(Ld, LSE[:, :, L - 1]) < 1e-13
+
+
+def test_attended_pairs_counts():
+    S = np.zeros((1, 1, 4, 4))
+    # train: history 0+1+2+3 blocks of 4x4 plus 4 triangles of 10
+    assert oracle.attended_pairs(S, 16, 4)[0, 0] == 6 * 16 + 4 * 10
+    assert oracle.attended_pairs(S, 16, 4, mode=oracle.SPARSE, topk=1)[0, 0] == 3 * 16 + 4 * 10
+
+
+# ------------------------------------------------------------- planted mistakes
+
+def _mutant(old, new):
+    """A fresh copy of the oracle module with one source substitution applied."""
+    src = inspect.getsource(ga)
+    assert src.count(old) == 1, old
+    ns = {"__name__": "oracle_mutant"}
+    exec(compile(src.replace(old, new), "<oracle mutant>", "exec"), ns)
+    return types.SimpleNamespace(**ns)
+
+
+def test_pins_catch_dropped_gate_term():
+    m = _mutant("gs - g_att * gs.sum()", "gs")
+    Q, K, V, S, W = _rand(5, 1, 2, 1, 32, 8, 4)
+    assert _fd_check(Q, K, V, S, 4, W, bwd=m.gated_attention_backward) > 1e-3
+
+
+def test_pins_catch_sign_error_in_softmax_jacobian():
+    m = _mutant("dz = p * (dp - np.sum(p * dp, axis=1, keepdims=True))",
+                "dz = p * (dp + np.sum(p * dp, axis=1, keepdims=True))")
+    Q, K, V, S, W = _rand(5, 1, 2, 1, 32, 8, 4)
+    assert _fd_check(Q, K, V, S, 4, W, bwd=m.gated_attention_backward) > 1e-3
+
+
+def test_pins_catch_unnormalised_gate():
+    m = _mutant("return s[A] - _logsumexp(s[norm_set])", "return s[A]")
+    Q = np.zeros((1, 1, 3, 1)); K = np.zeros((1, 1, 3, 1))
+    V = np.array([1.0, 2.0, 3.0]).reshape(1, 1, 3, 1)
+    S = np.zeros((1, 1, 3, 3)); S[0, 0, 2, 0] = math.log(3.0)
+    O, _ = m.gated_attention_forward(Q, K, V, S, 1)
+    assert abs(O[0, 0, 2, 0] - 17.0 / 8.0) > 1e-3
+
+
+def test_pins_catch_current_block_in_history():
+    m = _mutant("return np.arange(r, dtype=np.int64)", "return np.arange(r + 1, dtype=np.int64)")
+    Q, K, V, S, _ = _rand(1, 1, 2, 2, 64, 16, 16)
+    O, _ = m.gated_attention_forward(Q, K, V, S, 16, gate="ones")
+    O_ref, _ = sdpa_dense_causal(Q, K, V)
+    assert rel_err(O, O_ref) > 1e-3
