@@ -1,0 +1,176 @@
+"""Thin ctypes binding over libgbs.so (the C ABI in include/gbs.h).
+
+Argument marshalling only: torch tensors supply device memory and the current
+stream; every step of the computation runs in the library's CUDA kernels.
+There is no fallback: if the library or a CUDA device is missing, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libgbs.so")
+
+GBS_OK = 0
+STATUS_NAMES = {0: "GBS_OK", 1: "GBS_ERR_INVALID_ARG", 2: "GBS_ERR_UNSUPPORTED", 3: "GBS_ERR_CUDA",
+                4: "GBS_ERR_TIMEOUT", 5: "GBS_ERR_WORKSPACE"}
+MODES = {"train": 0, "sparse": 1}
+DTYPES = {torch.bfloat16: 0, torch.float32: 1}
+OP_FWD, OP_BWD, OP_DECODE = 0, 1, 2
+
+EXPORTED = ("gbs_version", "gbs_status_string", "gbs_last_error", "gbs_workspace_bytes",
+            "gbs_clear_error", "gbs_check", "gbs_select", "gbs_fwd", "gbs_bwd", "gbs_decode")
+
+
+class GbsError(RuntimeError):
+    def __init__(self, status, where, detail=""):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} {detail}".strip())
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("N", ctypes.c_int), ("d", ctypes.c_int), ("block", ctypes.c_int),
+                ("topk", ctypes.c_int), ("mode", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("scale", ctypes.c_float)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Loads libgbs.so and declares the argument types of every entry point."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing; build it with gated_block_sparse_gate_b200.build")
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER(Params)
+    vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    sigs = {
+        "gbs_version": (i32, []),
+        "gbs_status_string": (ctypes.c_char_p, [i32]),
+        "gbs_last_error": (ctypes.c_char_p, []),
+        "gbs_workspace_bytes": (sz, [P, i32]),
+        "gbs_clear_error": (i32, [vp, vp]),
+        "gbs_check": (i32, [vp, vp]),
+        "gbs_select": (i32, [P, vp, vp, vp, vp, vp, vp]),
+        "gbs_fwd": (i32, [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "gbs_bwd": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "gbs_decode": (i32, [P, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]),
+    }
+    for name, (res, args) in sigs.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(status, where):
+    if status != GBS_OK:
+        detail = load_library().gbs_last_error().decode()
+        raise GbsError(status, where, detail)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_params(B, Hq, Hkv, N, d, block=64, topk=0, mode="train", dtype=torch.bfloat16, scale=0.0):
+    return Params(B, Hq, Hkv, N, d, block, topk, MODES[mode], DTYPES[dtype], float(scale))
+
+
+def workspace_bytes(params: Params, op: int) -> int:
+    return int(load_library().gbs_workspace_bytes(ctypes.byref(params), op))
+
+
+def alloc_workspace(params: Params, op: int, device) -> torch.Tensor:
+    n = workspace_bytes(params, op)
+    if n == 0:
+        raise GbsError(1, "workspace_bytes", load_library().gbs_last_error().decode())
+    ws = torch.zeros(n, dtype=torch.uint8, device=device)
+    assert ws.data_ptr() % 256 == 0
+    return ws
+
+
+def _prefill_params(Q, K, S, block, topk, mode, scale):
+    B, Hq, N, d = Q.shape
+    return make_params(B, Hq, K.shape[1], N, d, block, topk, mode, Q.dtype, scale)
+
+
+def select(S, block=64, topk=0, mode="sparse", N=None, stream=None):
+    """K1: (idx, cnt, logg, slse) for S [B, Hq, Nb, Nb]."""
+    lib = load_library()
+    B, Hq, Nb, _ = S.shape
+    N = N if N is not None else Nb * block
+    p = make_params(B, Hq, Hq, N, 64, block, topk, mode, torch.float32)
+    dev = S.device
+    idx = cnt = logg = None
+    if mode == "sparse":
+        idx = torch.empty(B, Hq, Nb, topk, dtype=torch.int32, device=dev)
+        cnt = torch.empty(B, Hq, Nb, dtype=torch.int32, device=dev)
+        logg = torch.empty(B, Hq, Nb, topk, dtype=torch.float32, device=dev)
+    slse = torch.empty(B, Hq, Nb, dtype=torch.float32, device=dev)
+    _check(lib.gbs_select(ctypes.byref(p), _ptr(S), _ptr(idx), _ptr(cnt), _ptr(logg), _ptr(slse),
+                          _stream(stream)), "gbs_select")
+    return idx, cnt, logg, slse
+
+
+def forward(Q, K, V, S, block=64, mode="train", topk=0, scale=0.0, out=None, lse=None, ws=None,
+            stream=None):
+    """Gated attention forward: returns (O, LSE)."""
+    lib = load_library()
+    p = _prefill_params(Q, K, S, block, topk, mode, scale)
+    O = out if out is not None else torch.empty_like(Q)
+    LSE = lse if lse is not None else torch.empty(Q.shape[:3], dtype=torch.float32, device=Q.device)
+    if ws is None:
+        ws = alloc_workspace(p, OP_FWD, Q.device)
+    _check(lib.gbs_fwd(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(S), _ptr(O), _ptr(LSE),
+                       _ptr(ws), ws.numel(), _stream(stream)), "gbs_fwd")
+    return O, LSE
+
+
+def backward(Q, K, V, S, O, LSE, dO, block=64, scale=0.0, grads=None, ws=None, stream=None):
+    """Training-mode backward: returns (dQ, dK, dV, dS)."""
+    lib = load_library()
+    p = _prefill_params(Q, K, S, block, 0, "train", scale)
+    if grads is None:
+        grads = (torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V), torch.empty_like(S))
+    dQ, dK, dV, dS = grads
+    if ws is None:
+        ws = alloc_workspace(p, OP_BWD, Q.device)
+    _check(lib.gbs_bwd(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(S), _ptr(O), _ptr(LSE),
+                       _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dS), _ptr(ws), ws.numel(),
+                       _stream(stream)), "gbs_bwd")
+    return dQ, dK, dV, dS
+
+
+def decode(q, Kc, Vc, S, L=None, block=64, topk=32, scale=0.0, num_splits=0, out=None, lse=None,
+           ws=None, stream=None):
+    """Sparse one-token decode: returns (O [B,Hq,d], LSE [B,Hq])."""
+    lib = load_library()
+    B, Hq, d = q.shape
+    L = Kc.shape[2] if L is None else L
+    p = make_params(B, Hq, Kc.shape[1], L, d, block, topk, "sparse", q.dtype, scale)
+    O = out if out is not None else torch.empty_like(q)
+    LSE = lse if lse is not None else torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = alloc_workspace(p, OP_DECODE, q.device)
+    _check(lib.gbs_decode(ctypes.byref(p), _ptr(q), _ptr(Kc), _ptr(Vc), _ptr(S), _ptr(O), _ptr(LSE),
+                          num_splits, _ptr(ws), ws.numel(), _stream(stream)), "gbs_decode")
+    return O, LSE
+
+
+def check(ws, stream=None):
+    """Raises GbsError if a kernel recorded a device-side error in ``ws``."""
+    _check(load_library().gbs_check(_ptr(ws), _stream(stream)), "gbs_check")

@@ -1,0 +1,223 @@
+// decode.cu — K4: sparse one-token decode, split over the selected blocks.
+//
+// One query per sequence sits at position L-1; its current block
+// cur = (L-1)/64 is always attended (bias 0, keys up to L-1) and the historical
+// blocks are the Top-K list of K1 with gates renormalised over it (NeurIPS
+// 2026 poster page of "SAS: Simple Attention Sparsification via End-to-End
+// Optimization of Context Ranking", Abstract: a fixed budget of context units
+// per query; Hugging Face paper page, Abstract: the current block is always
+// retained).
+//
+// The work is bound by HBM: every selected block streams 64 keys and 64 values
+// once. Split kernel: grid (B*Hq, splits); each CTA takes a contiguous share of
+// the (selected + current) block list; a group of D/8 lanes owns one key row
+// and loads it with 16-byte vector loads (eight loads in flight per lane before
+// any arithmetic), reduces the dot product with shuffles and keeps an online
+// softmax state. The CTA merges its eight groups and writes one partial
+// (m, l, acc[D]) per split; the combine kernel merges the splits.
+#include "common.cuh"
+#include "internal.h"
+
+namespace gbs {
+
+namespace {
+
+constexpr int kBS = 64;
+constexpr int kThreads = 128;
+
+struct Vec8 {
+  float v[8];
+};
+
+template <typename T>
+__device__ __forceinline__ Vec8 load8(const T* ptr);
+
+template <>
+__device__ __forceinline__ Vec8 load8<__nv_bfloat16>(const __nv_bfloat16* ptr) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(ptr));
+  Vec8 r;
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    r.v[2 * i] = f.x;
+    r.v[2 * i + 1] = f.y;
+  }
+  return r;
+}
+
+template <>
+__device__ __forceinline__ Vec8 load8<float>(const float* ptr) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(ptr));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(ptr) + 1);
+  Vec8 r;
+  r.v[0] = a.x; r.v[1] = a.y; r.v[2] = a.z; r.v[3] = a.w;
+  r.v[4] = b.x; r.v[5] = b.y; r.v[6] = b.z; r.v[7] = b.w;
+  return r;
+}
+
+// Online-softmax state of one lane group (log2 domain).
+struct State {
+  float m, l, acc[8];
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads)
+decode_split_kernel(Problem p, const T* __restrict__ q, const T* __restrict__ Kc,
+                    const T* __restrict__ Vc, Selection sel, int cur, int splits,
+                    float* __restrict__ part_ml, float* __restrict__ part_acc) {
+  constexpr int LPK = D / 8;             // lanes per key row
+  constexpr int GPW = 32 / LPK;          // key groups per warp
+  constexpr int NGROUPS = (kThreads / 32) * GPW;
+  constexpr int ROWS_PER_GROUP = kBS / NGROUPS;
+  __shared__ float s_m[NGROUPS], s_l[NGROUPS];
+  __shared__ float s_acc[NGROUPS][D];
+
+  const int bh = blockIdx.x, split = blockIdx.y;
+  const int b = bh / p.Hq, h = bh % p.Hq, kvh = h / p.G;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp_in_warp = lane / LPK, sub = lane % LPK;
+  const int group = warp * GPW + grp_in_warp;
+  const int n_hist = sel.cnt[bh];
+  const int n_ent = n_hist + 1;  // + current block
+  const int per = (n_ent + splits - 1) / splits;
+  const int e0 = split * per, e1 = min(n_ent, e0 + per);
+  const int L = p.N;
+
+  Vec8 qv = load8<T>(q + (size_t)bh * D + sub * 8);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) qv.v[i] *= p.scale_log2;
+
+  State st;
+  st.m = -INFINITY;
+  st.l = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) st.acc[i] = 0.f;
+
+  const size_t kvbase = ((size_t)(b * p.Hkv + kvh) * L) * D;
+  for (int e = e0; e < e1; ++e) {
+    const bool is_cur = e == n_hist;
+    const int c = is_cur ? cur : sel.idx[(size_t)bh * p.topk + e];
+    const float bias2 = is_cur ? 0.f : sel.logg[(size_t)bh * p.topk + e] * GBS_LOG2E;
+    // rows handled by this group inside the block
+    const int row0 = c * kBS + group * ROWS_PER_GROUP;
+    Vec8 kv[ROWS_PER_GROUP];
+    float s[ROWS_PER_GROUP];
+#pragma unroll
+    for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) {
+      const int row = min(row0 + rr, L - 1);
+      kv[rr] = load8<T>(Kc + kvbase + (size_t)row * D + sub * 8);
+    }
+#pragma unroll
+    for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) {
+      float d = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) d = fmaf(qv.v[i], kv[rr].v[i], d);
+#pragma unroll
+      for (int o = LPK / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+      s[rr] = (row0 + rr < L) ? d + bias2 : -INFINITY;
+    }
+#pragma unroll
+    for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) {
+      const int row = min(row0 + rr, L - 1);
+      kv[rr] = load8<T>(Vc + kvbase + (size_t)row * D + sub * 8);
+    }
+    float mloc = st.m;
+#pragma unroll
+    for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) mloc = fmaxf(mloc, s[rr]);
+    if (mloc > -INFINITY) {
+      const float corr = exp2f(st.m - mloc);
+      st.l *= corr;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) st.acc[i] *= corr;
+      st.m = mloc;
+#pragma unroll
+      for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) {
+        const float pr = exp2f(s[rr] - mloc);
+        st.l += pr;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) st.acc[i] = fmaf(pr, kv[rr].v[i], st.acc[i]);
+      }
+    }
+  }
+  // merge the groups of the CTA
+  if (sub == 0) {
+    s_m[group] = st.m;
+    s_l[group] = st.l;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) s_acc[group][sub * 8 + i] = st.acc[i];
+  __syncthreads();
+  float M = -INFINITY;
+#pragma unroll
+  for (int g = 0; g < NGROUPS; ++g) M = fmaxf(M, s_m[g]);
+  const size_t pidx = (size_t)bh * splits + split;
+  for (int k = threadIdx.x; k < D; k += kThreads) {
+    float a = 0.f;
+    if (M > -INFINITY)
+      for (int g = 0; g < NGROUPS; ++g) a += s_acc[g][k] * exp2f(s_m[g] - M);
+    part_acc[pidx * D + k] = a;
+  }
+  if (threadIdx.x == 0) {
+    float l = 0.f;
+    if (M > -INFINITY)
+      for (int g = 0; g < NGROUPS; ++g) l += s_l[g] * exp2f(s_m[g] - M);
+    part_ml[pidx * 2] = M;
+    part_ml[pidx * 2 + 1] = l;
+  }
+}
+
+template <typename T, int D>
+__global__ void decode_combine_kernel(Problem p, int splits, const float* __restrict__ part_ml,
+                                      const float* __restrict__ part_acc, T* __restrict__ O,
+                                      float* __restrict__ LSE) {
+  const int bh = blockIdx.x;
+  float M = -INFINITY;
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, part_ml[((size_t)bh * splits + s) * 2]);
+  float l = 0.f;
+  for (int s = 0; s < splits; ++s) {
+    const float ms = part_ml[((size_t)bh * splits + s) * 2];
+    if (ms > -INFINITY) l += part_ml[((size_t)bh * splits + s) * 2 + 1] * exp2f(ms - M);
+  }
+  const float inv = 1.f / l;
+  for (int k = threadIdx.x; k < D; k += blockDim.x) {
+    float a = 0.f;
+    for (int s = 0; s < splits; ++s) {
+      const float ms = part_ml[((size_t)bh * splits + s) * 2];
+      if (ms > -INFINITY) a += part_acc[((size_t)bh * splits + s) * D + k] * exp2f(ms - M);
+    }
+    O[(size_t)bh * D + k] = from_f32<T>(a * inv);
+  }
+  if (threadIdx.x == 0) LSE[bh] = (M + log2f(l)) * GBS_LN2;
+}
+
+template <typename T, int D>
+cudaError_t decode_typed(const Problem& p, const void* q, const void* Kc, const void* Vc,
+                         const Selection& sel, int cur, int splits, float* part_ml,
+                         float* part_acc, void* O, float* LSE, cudaStream_t st) {
+  const int BH = p.B * p.Hq;
+  decode_split_kernel<T, D><<<dim3(BH, splits), kThreads, 0, st>>>(
+      p, (const T*)q, (const T*)Kc, (const T*)Vc, sel, cur, splits, part_ml, part_acc);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_combine_kernel<T, D><<<BH, D, 0, st>>>(p, splits, part_ml, part_acc, (T*)O, LSE);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const Problem& p, const void* q, const void* Kc, const void* Vc,
+                          const Selection& sel, int cur, int num_splits, float* part_ml,
+                          float* part_acc, void* O, float* LSE, cudaStream_t st) {
+  if (p.bs != kBS) return cudaErrorNotSupported;
+  if (p.dtype == GBS_F32) {
+    if (p.d == 64) return decode_typed<float, 64>(p, q, Kc, Vc, sel, cur, num_splits, part_ml, part_acc, O, LSE, st);
+    if (p.d == 128) return decode_typed<float, 128>(p, q, Kc, Vc, sel, cur, num_splits, part_ml, part_acc, O, LSE, st);
+  } else {
+    if (p.d == 64) return decode_typed<__nv_bfloat16, 64>(p, q, Kc, Vc, sel, cur, num_splits, part_ml, part_acc, O, LSE, st);
+    if (p.d == 128) return decode_typed<__nv_bfloat16, 128>(p, q, Kc, Vc, sel, cur, num_splits, part_ml, part_acc, O, LSE, st);
+  }
+  return cudaErrorNotSupported;
+}
+
+}  // namespace gbs

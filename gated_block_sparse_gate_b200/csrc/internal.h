@@ -1,0 +1,56 @@
+// internal.h — launchers shared between the C ABI (gbs_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "gbs.h"
+
+namespace gbs {
+
+// Resolved problem description handed to every launcher.
+struct Problem {
+  int B, Hq, Hkv, N, d, bs, Nb, G, topk, mode, dtype;
+  float scale;        // logit scale (natural units)
+  float scale_log2;   // scale * log2(e)
+};
+
+// Selection buffers produced by K1 and read by the attention kernels.
+struct Selection {
+  float* slse;     // [B, Hq, Nb]   training normaliser (may be null in sparse mode)
+  int32_t* idx;    // [B, Hq, Nb, topk] (sparse only)
+  int32_t* cnt;    // [B, Hq, Nb]
+  float* logg;     // [B, Hq, Nb, topk]
+};
+
+// K1: gate normalisation (+ Top-K in sparse mode). rows_per_head = Nb for
+// prefill/training (row r has history r); for decode rows_per_head = 1 and
+// every row has history `decode_cur`.
+cudaError_t launch_select(const float* S, int n_rows, int row_stride, int rows_per_head,
+                          int decode_cur, int topk, bool sparse, int32_t* idx, int32_t* cnt,
+                          float* logg, float* slse, cudaStream_t st);
+
+// Exact SIMT path (fp32 math for fp32 or bf16 storage).
+cudaError_t launch_fwd_simt(const Problem& p, const void* Q, const void* K, const void* V,
+                            const float* S, const Selection& sel, void* O, float* LSE,
+                            cudaStream_t st);
+cudaError_t launch_bwd_simt(const Problem& p, const void* Q, const void* K, const void* V,
+                            const float* S, const float* slse, const void* O, const float* LSE,
+                            const void* dO, void* dQ, void* dK, void* dV, float* dS,
+                            float* Dvec, float* Gblk, cudaStream_t st);
+
+// Decode (split over the selected blocks, then combine).
+cudaError_t launch_decode(const Problem& p, const void* q, const void* Kc, const void* Vc,
+                          const Selection& sel, int cur, int num_splits, float* part_ml,
+                          float* part_acc, void* O, float* LSE, cudaStream_t st);
+
+// Tensor-core path (sm_100a, bf16). Returns cudaErrorNotSupported when the
+// configuration is outside what the kernel handles.
+cudaError_t launch_fwd_tc(const Problem& p, const void* Q, const void* K, const void* V,
+                          const float* S, const Selection& sel, const int32_t* plan,
+                          int plan_stride, void* O, float* LSE, unsigned int* err,
+                          cudaStream_t st);
+bool fwd_tc_supported(const Problem& p);
+
+}  // namespace gbs

@@ -1,0 +1,133 @@
+// select.cu — K1: gate normalisation and Top-K block selection.
+//
+// Normalised softmax gates in log form (Hugging Face paper page of "SAS: Simple
+// Attention Sparsification via End-to-End Optimization of Context Ranking",
+// Abstract; ai.viyan.live blog, section "Differentiable Budget Constraints"),
+// and the fixed-budget hard Top-K used at inference (NeurIPS 2026 poster page,
+// Abstract).
+//
+// One warp owns one score row. Training mode only needs the row's log-sum-exp
+// over the historical blocks c < r. Sparse mode finds the K-th largest score by
+// a most-significant-bit-first threshold search on order-preserving 32-bit
+// keys (32 counting passes over the row in shared memory), keeps every block
+// above the threshold plus the lowest-index blocks equal to it, compacts them
+// in ascending index order with ballots, and renormalises the log gates over
+// the kept set. Comparisons are exact on the fp32 scores, so the index lists
+// are bit-identical to any other exact implementation of the same ordering.
+#include "common.cuh"
+#include "internal.h"
+
+namespace gbs {
+
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kRowCache = 2048;  // scores cached in shared memory per warp
+
+__device__ __forceinline__ float row_score(const float* srow, const uint32_t* cache, bool cached,
+                                           int c) {
+  return cached ? __uint_as_float(cache[c]) : __ldg(srow + c);
+}
+
+__global__ void __launch_bounds__(kWarps * 32)
+select_kernel(const float* __restrict__ S, int n_rows, int row_stride, int rows_per_head,
+              int decode_cur, int topk, int sparse, int32_t* __restrict__ idx,
+              int32_t* __restrict__ cnt, float* __restrict__ logg, float* __restrict__ slse) {
+  __shared__ uint32_t cache_all[kWarps][kRowCache];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * kWarps + warp;
+  if (row >= n_rows) return;
+  const int r = decode_cur >= 0 ? decode_cur : (row % rows_per_head);
+  const float* srow = S + (size_t)row * row_stride;
+  uint32_t* cache = cache_all[warp];
+  const bool cached = r <= kRowCache;
+  if (cached)
+    for (int c = lane; c < r; c += 32) cache[c] = __float_as_uint(__ldg(srow + c));
+  __syncwarp();
+
+  // Training-mode normaliser over all of H_r.
+  if (slse) {
+    float m = -INFINITY;
+    for (int c = lane; c < r; c += 32) m = fmaxf(m, row_score(srow, cache, cached, c));
+    m = warp_max(m);
+    float s = 0.f;
+    for (int c = lane; c < r; c += 32) s += expf(row_score(srow, cache, cached, c) - m);
+    s = warp_sum(s);
+    if (lane == 0) slse[row] = r > 0 ? m + logf(s) : -INFINITY;
+  }
+  if (!sparse) return;
+
+  const int k = min(topk, r);
+  int32_t* out_idx = idx + (size_t)row * topk;
+  float* out_logg = logg + (size_t)row * topk;
+
+  // Threshold T = the k-th largest key; count_ge(T) >= k and count_gt(T) < k.
+  uint32_t T = 0u;
+  int need_eq = 0;
+  if (k > 0 && k < r) {
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = T | (1u << bit);
+      int n = 0;
+      for (int c = lane; c < r; c += 32) n += ordered_key(row_score(srow, cache, cached, c)) >= cand;
+      n = __reduce_add_sync(0xffffffffu, n);
+      if (n >= k) T = cand;
+    }
+    int gt = 0;
+    for (int c = lane; c < r; c += 32) gt += ordered_key(row_score(srow, cache, cached, c)) > T;
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    need_eq = k - gt;
+  }
+
+  // Compact the kept blocks in ascending index order.
+  int written = 0, eq_seen = 0;
+  float m = -INFINITY;
+  const uint32_t lanes_below = (1u << lane) - 1u;
+  for (int base = 0; base < r && written < k; base += 32) {
+    const int c = base + lane;
+    const bool valid = c < r;
+    const float s = valid ? row_score(srow, cache, cached, c) : 0.f;
+    const uint32_t u = ordered_key(s);
+    const bool eq = valid && k < r && u == T;
+    const uint32_t eq_mask = __ballot_sync(0xffffffffu, eq);
+    const int eq_before = eq_seen + __popc(eq_mask & lanes_below);
+    const bool keep = valid && (k >= r || u > T || (eq && eq_before < need_eq));
+    eq_seen += __popc(eq_mask);
+    const uint32_t keep_mask = __ballot_sync(0xffffffffu, keep);
+    const int pos = written + __popc(keep_mask & lanes_below);
+    if (keep) {
+      out_idx[pos] = c;
+      out_logg[pos] = s;  // raw score for now, normalised below
+      m = fmaxf(m, s);
+    }
+    written += __popc(keep_mask);
+  }
+  __syncwarp();
+  m = warp_max(m);
+  float sum = 0.f;
+  for (int j = lane; j < k; j += 32) sum += expf(out_logg[j] - m);
+  sum = warp_sum(sum);
+  const float lse = m + logf(sum);
+  for (int j = lane; j < topk; j += 32) {
+    if (j < k) {
+      out_logg[j] = out_logg[j] - lse;
+    } else {
+      out_idx[j] = -1;
+      out_logg[j] = 0.f;
+    }
+  }
+  if (lane == 0) cnt[row] = k;
+}
+
+}  // namespace
+
+cudaError_t launch_select(const float* S, int n_rows, int row_stride, int rows_per_head,
+                          int decode_cur, int topk, bool sparse, int32_t* idx, int32_t* cnt,
+                          float* logg, float* slse, cudaStream_t st) {
+  if (n_rows <= 0) return cudaSuccess;
+  const int grid = (n_rows + kWarps - 1) / kWarps;
+  select_kernel<<<grid, kWarps * 32, 0, st>>>(S, n_rows, row_stride, rows_per_head, decode_cur,
+                                              topk, sparse ? 1 : 0, idx, cnt, logg, slse);
+  return cudaGetLastError();
+}
+
+}  // namespace gbs

@@ -1,0 +1,163 @@
+/*
+ * gbs.h — C ABI of the gated block-sparse causal attention library (libgbs.so).
+ *
+ * The operation (SAS, "Simple Attention Sparsification via End-to-End
+ * Optimization of Context Ranking"):
+ *   - selector scores S over earlier key blocks become normalised softmax gates
+ *     g, applied in log form inside the attention softmax (NeurIPS 2026 poster
+ *     page, Abstract; Hugging Face paper page, Abstract);
+ *   - logit z_ij = scale * q_i.k_j + log g[r(i), c(j)] for keys in an attended
+ *     historical block c < r, + 0 for keys of the always-retained current block
+ *     r with j <= i, and -inf otherwise (ai.viyan.live, "SAS Learns Token
+ *     Importance for Sparse Attention", section "The Logit Injection Mechanism");
+ *   - training mode attends every historical block and the backward pass
+ *     returns dQ, dK, dV and dS, the gradient through the gate softmax into the
+ *     scores (same blog page and section; poster Abstract: all context units
+ *     active during training);
+ *   - sparse mode attends only the Top-K historical blocks by score plus the
+ *     current block (poster Abstract: fixed attention budget; HF page Abstract:
+ *     hard Top-K). Gates are renormalised over the selected blocks.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers (cudaMalloc / torch memory),
+ *     contiguous row-major in the layouts given per function, 16-byte aligned.
+ *     The caller owns every buffer, including the workspace `ws`; the library
+ *     never allocates, frees or synchronises (gbs_check excepted).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Work is
+ *     enqueued asynchronously.
+ *   - Arguments are validated before any launch; on failure the function
+ *     returns a status and leaves every output untouched; gbs_last_error()
+ *     then describes the failing argument.
+ *   - Launch failures return GBS_ERR_CUDA. Errors detected on the device
+ *     (a bounded wait that expired) are recorded in the workspace's error word
+ *     and reported by gbs_check().
+ *   - Layouts: Q, O, dO, dQ [B, Hq, N, d]; K, V, dK, dV [B, Hkv, N, d];
+ *     LSE [B, Hq, N] fp32; S, dS [B, Hq, Nb, Nb] fp32 with Nb = N / block
+ *     (only entries with c < r are read; dS is written 0 elsewhere).
+ *     q-head h reads kv-head h / (Hq / Hkv).
+ *   - Supported: d in {64, 128}; block == 64; N % 64 == 0 (training/prefill);
+ *     Hq % Hkv == 0; 0 <= topk <= GBS_MAX_TOPK; dtype bf16 (tensor-core path)
+ *     or fp32 (exact SIMT path). S must be finite.
+ */
+#ifndef GBS_H_
+#define GBS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GBS_API __attribute__((visibility("default")))
+#else
+#define GBS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GBS_VERSION_MAJOR 0
+#define GBS_VERSION_MINOR 1
+#define GBS_MAX_TOPK 256
+
+typedef enum gbs_status {
+  GBS_OK = 0,
+  GBS_ERR_INVALID_ARG = 1,   /* a shape, pointer, alignment or size is invalid  */
+  GBS_ERR_UNSUPPORTED = 2,   /* valid, but not a configuration this build runs  */
+  GBS_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed     */
+  GBS_ERR_TIMEOUT = 4,       /* a device-side bounded wait expired (gbs_check)  */
+  GBS_ERR_WORKSPACE = 5      /* workspace missing or smaller than required      */
+} gbs_status;
+
+typedef enum gbs_mode { GBS_TRAIN = 0, GBS_SPARSE = 1 } gbs_mode;
+typedef enum gbs_dtype { GBS_BF16 = 0, GBS_F32 = 1 } gbs_dtype;
+typedef enum gbs_op { GBS_OP_FWD = 0, GBS_OP_BWD = 1, GBS_OP_DECODE = 2 } gbs_op;
+
+typedef struct gbs_params {
+  int B;        /* batch                                                     */
+  int Hq;       /* query heads                                               */
+  int Hkv;      /* key/value heads, Hq % Hkv == 0                            */
+  int N;        /* tokens (training / prefill) or cache length L (decode)   */
+  int d;        /* head dimension                                            */
+  int block;    /* context-unit block size (tokens per block)               */
+  int topk;     /* sparse budget K of historical blocks (sparse / decode)   */
+  int mode;     /* gbs_mode                                                  */
+  int dtype;    /* gbs_dtype of Q, K, V, O, dO, dQ, dK, dV                   */
+  float scale;  /* logit scale; 0 selects 1/sqrt(d)                          */
+} gbs_params;
+
+/* Version as (major << 16) | minor. */
+GBS_API int gbs_version(void);
+
+/* Text of a status code; never NULL. */
+GBS_API const char* gbs_status_string(gbs_status s);
+
+/* Description of the last validation failure on the calling thread ("" if none). */
+GBS_API const char* gbs_last_error(void);
+
+/* Bytes of workspace `ws` that gbs_fwd / gbs_bwd / gbs_decode need for `op`
+ * with these parameters (0 if the parameters are invalid). The workspace must
+ * be device memory, 256-byte aligned, and must not be shared by calls that run
+ * concurrently. Its first word is the device error word read by gbs_check. */
+GBS_API size_t gbs_workspace_bytes(const gbs_params* p, int op);
+
+/* Clears the device error word of `ws` (asynchronous, on `stream`). */
+GBS_API gbs_status gbs_clear_error(void* ws, void* stream);
+
+/* Reads the device error word of `ws`: synchronises `stream`, returns GBS_OK
+ * or the recorded status (GBS_ERR_TIMEOUT when a bounded wait expired). */
+GBS_API gbs_status gbs_check(const void* ws, void* stream);
+
+/* Gate normalisation and Top-K block selection (K1).
+ * Normalised softmax gates in log form over the attended historical set
+ * (HF page Abstract; blog section "Differentiable Budget Constraints").
+ *   S     [B, Hq, Nb, Nb] fp32, row r scores key blocks c < r.
+ *   slse  [B, Hq, Nb] fp32 out: ln sum_{c<r} exp S[r, c] (-inf for r = 0);
+ *         may be NULL in sparse mode.
+ *   Sparse mode only (may be NULL in training mode):
+ *   idx   [B, Hq, Nb, topk] int32 out: A_r ascending, -1 padded. A_r holds the
+ *         min(topk, r) blocks c < r with the largest S[r, c]; ties go to the
+ *         lower index; -0.0 equals +0.0.
+ *   cnt   [B, Hq, Nb] int32 out: |A_r|.
+ *   logg  [B, Hq, Nb, topk] fp32 out: S[r, c] - ln sum_{c' in A_r} exp S[r, c'],
+ *         0 in the padding. */
+GBS_API gbs_status gbs_select(const gbs_params* p, const float* S, int32_t* idx, int32_t* cnt,
+                      float* logg, float* slse, void* stream);
+
+/* Gated attention forward (select + attention).
+ *   Q [B,Hq,N,d], K/V [B,Hkv,N,d] in p->dtype; S [B,Hq,Nb,Nb] fp32.
+ *   O [B,Hq,N,d] out (p->dtype); LSE [B,Hq,N] fp32 out, natural log of
+ *   sum_j exp z_ij with z including scale and bias.
+ *   p->mode selects training (every block c < r, gates over all of them) or
+ *   sparse (Top-K blocks, gates renormalised over them).
+ *   ws: gbs_workspace_bytes(p, GBS_OP_FWD) bytes. */
+GBS_API gbs_status gbs_fwd(const gbs_params* p, const void* Q, const void* K, const void* V,
+                   const float* S, void* O, float* LSE, void* ws, size_t ws_bytes,
+                   void* stream);
+
+/* Gated attention backward, training mode (p->mode must be GBS_TRAIN).
+ *   O, LSE: outputs of gbs_fwd for the same inputs. dO [B,Hq,N,d] (p->dtype).
+ *   dQ [B,Hq,N,d], dK/dV [B,Hkv,N,d] out (p->dtype; fp32 accumulation).
+ *   dS [B,Hq,Nb,Nb] fp32 out: dS[r,c'] = G[r,c'] - g[r,c'] sum_{c<r} G[r,c]
+ *   for c' < r and 0 elsewhere, where G[r,c] sums dL/dz over the (r,c) tile.
+ *   ws: gbs_workspace_bytes(p, GBS_OP_BWD) bytes. */
+GBS_API gbs_status gbs_bwd(const gbs_params* p, const void* Q, const void* K, const void* V,
+                   const float* S, const void* O, const float* LSE, const void* dO,
+                   void* dQ, void* dK, void* dV, float* dS, void* ws, size_t ws_bytes,
+                   void* stream);
+
+/* Sparse decode: one query per sequence at position L-1 (L = p->N).
+ *   q [B,Hq,d]; Kc/Vc [B,Hkv,L,d] (p->dtype); S [B,Hq,Nb] fp32 with
+ *   Nb = ceil(L / block): scores of the current block's row over key blocks
+ *   c < cur = (L-1)/block. Attends the Top-K (p->topk) historical blocks with
+ *   renormalised log gates plus the current block up to L-1 with bias 0.
+ *   O [B,Hq,d] out (p->dtype); LSE [B,Hq] fp32 out.
+ *   num_splits: partitions of the selected blocks per (b, h); 0 = automatic.
+ *   ws: gbs_workspace_bytes(p, GBS_OP_DECODE) bytes. */
+GBS_API gbs_status gbs_decode(const gbs_params* p, const void* q, const void* Kc, const void* Vc,
+                      const float* S, void* O, float* LSE, int num_splits, void* ws,
+                      size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GBS_H_ */

@@ -1,0 +1,232 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 oracle.
+
+Tolerances (normwise relative, max|x - ref| / max|ref|): O and LSE 1e-5 for
+fp32 and 2e-2 for bf16; gradients 5e-2; block index lists bit-exact.
+Full-size workloads are checked on sampled rows / kv-groups / sequences that
+the oracle computes one by one, in the launch configuration the bench times.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_block_sparse_gate_b200 import binding as gb
+from gated_block_sparse_gate_b200.build import build
+from gated_block_sparse_gate_b200.inputs import WORKLOADS, make_decode_inputs, make_prefill_inputs
+from tests.oracle_refs import rel_err
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-5
+TOL_BF16 = 2e-2
+TOL_GRAD = 5e-2
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build()
+    gb.load_library()
+
+
+def np64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def _small(seed, B, Hq, Hkv, N, d, dtype, scaled, with_grad=True):
+    g = torch.Generator().manual_seed(seed)
+    scl = d ** -0.5 if scaled else 1.0
+    Q = (torch.randn(B, Hq, N, d, generator=g) * scl).to(dtype)
+    K = (torch.randn(B, Hkv, N, d, generator=g) * scl).to(dtype)
+    V = (torch.randn(B, Hkv, N, d, generator=g) * scl).to(dtype)
+    S = torch.randn(B, Hq, N // 64, N // 64, generator=g) * math.sqrt(2)
+    dO = torch.randn(B, Hq, N, d, generator=g).to(dtype)
+    return dict(Q=Q, K=K, V=V, S=S, dO=dO)
+
+
+def _dev(x):
+    return {k: v.to(DEV) for k, v in x.items()}
+
+
+# ------------------------------------------------------------------- selection
+
+def test_select_tiny_workload_bit_exact():
+    w = WORKLOADS["tiny_f32_n1024"]
+    S = make_prefill_inputs(w)["S"]
+    for k in (0, 1, 4, 15, 16, 40):
+        idx, cnt, logg, slse = gb.select(S.to(DEV), topk=k, mode="sparse")
+        ri, rc, rl, rs = oracle.select_blocks(S.numpy(), 16, k)
+        assert np.array_equal(idx.cpu().numpy(), ri)
+        assert np.array_equal(cnt.cpu().numpy(), rc)
+        assert np.max(np.abs(logg.cpu().numpy() - rl), initial=0.0) < 1e-5
+    _, _, _, slse = gb.select(S.to(DEV), mode="train")
+    _, _, _, rs = oracle.select_blocks(S.numpy(), 16, None, mode=oracle.TRAIN)
+    fin = np.isfinite(rs)
+    assert np.array_equal(np.isfinite(slse.cpu().numpy()), fin)
+    assert np.max(np.abs(slse.cpu().numpy()[fin] - rs[fin])) < 1e-5
+
+
+def test_select_ties_and_signed_zero_bit_exact():
+    g = torch.Generator().manual_seed(123)
+    S = torch.randint(-2, 3, (2, 3, 70, 70), generator=g).float()
+    S[torch.rand(S.shape, generator=g) < 0.2] = -0.0
+    for k in (1, 3, 7, 33, 69, 200):
+        idx, cnt, _, _ = gb.select(S.to(DEV), topk=k, mode="sparse")
+        ri, rc, _, _ = oracle.select_blocks(S.numpy(), 70, k)
+        assert np.array_equal(idx.cpu().numpy(), ri), k
+        assert np.array_equal(cnt.cpu().numpy(), rc), k
+
+
+@pytest.mark.parametrize("k", [8, 16, 32, 64])
+def test_select_sparse_prefill_full_size_sampled(k):
+    """Planted-score workload (N=65536, 1024 blocks per row), sampled rows."""
+    w = WORKLOADS["sparse_prefill_bf16_n65536"]
+    S = make_prefill_inputs(w, with_grad=False)["S"]
+    idx, cnt, logg, _ = gb.select(S.to(DEV), topk=k, mode="sparse")
+    idx, cnt, logg = idx.cpu().numpy(), cnt.cpu().numpy(), logg.cpu().numpy()
+    rng = np.random.default_rng(k)
+    Sn = S.numpy()
+    for h in (0, 13, 31):
+        for r in list(rng.integers(0, 1024, 40)) + [0, 1, k - 1, k, k + 1, 1023]:
+            A = oracle.attended_blocks(Sn[0, h, r], r, oracle.SPARSE, k)
+            assert cnt[0, h, r] == len(A)
+            assert np.array_equal(idx[0, h, r, :len(A)], A)
+            assert np.all(idx[0, h, r, len(A):] == -1)
+            lg = oracle.log_gates(Sn[0, h, r], A, r)
+            assert np.max(np.abs(logg[0, h, r, :len(A)] - lg), initial=0) < 1e-5
+
+
+# ---------------------------------------------------------------------- forward
+
+def _check_fwd(x, mode, k, tol, rows=None):
+    Qd, Kd, Vd, Sd = (x[n].to(DEV) for n in "QKVS")
+    O, LSE = gb.forward(Qd, Kd, Vd, Sd, mode=mode, topk=k)
+    torch.cuda.synchronize()
+    Or, Lr = oracle.gated_attention_forward(np64(x["Q"]), np64(x["K"]), np64(x["V"]), x["S"].numpy(),
+                                            64, mode=mode, topk=k, rows=rows)
+    eo, el = rel_err(np64(O), Or), rel_err(LSE.cpu().numpy(), Lr)
+    assert eo < tol and el < tol, (eo, el)
+    return eo, el
+
+
+def test_fwd_tiny_f32_train_and_sparse():
+    x = make_prefill_inputs(WORKLOADS["tiny_f32_n1024"])
+    _check_fwd(x, "train", 0, TOL_F32)
+    _check_fwd(x, "sparse", 4, TOL_F32)
+
+
+@pytest.mark.parametrize("mode,k", [("train", 0), ("sparse", 0), ("sparse", 3), ("sparse", 100)])
+@pytest.mark.parametrize("scaled", [True, False])
+def test_fwd_bf16_small(mode, k, scaled):
+    x = _small(7, 1, 8, 2, 1024, 128, torch.bfloat16, scaled)
+    _check_fwd(x, mode, k, TOL_BF16)
+
+
+@pytest.mark.parametrize("shape", [
+    (1, 2, 2, 64, 128),    # one block: no history
+    (2, 4, 4, 320, 64),    # odd block count, MHA, d=64
+    (1, 4, 1, 448, 128),   # GQA 4:1, 7 blocks
+])
+@pytest.mark.parametrize("mode,k", [("train", 0), ("sparse", 2)])
+def test_fwd_edge_shapes(shape, mode, k):
+    B, Hq, Hkv, N, d = shape
+    for dtype, tol in ((torch.bfloat16, TOL_BF16), (torch.float32, TOL_F32)):
+        x = _small(11, B, Hq, Hkv, N, d, dtype, scaled=False)
+        _check_fwd(x, mode, k, tol)
+
+
+def test_fwd_train_full_size_sampled():
+    """Training workload N=8192, 32/8 heads, bf16: sampled query blocks."""
+    w = WORKLOADS["train_bf16_n8192"]
+    x = make_prefill_inputs(w, with_grad=False)
+    rows = [(0, h, r) for h in (0, 5, 31) for r in (0, 1, 2, 63, 64, 100, 126, 127)]
+    _check_fwd(x, "train", 0, TOL_BF16, rows=rows)
+
+
+@pytest.mark.parametrize("k", [8, 64])
+def test_fwd_sparse_prefill_full_size_sampled(k):
+    w = WORKLOADS["sparse_prefill_bf16_n65536"]
+    x = make_prefill_inputs(w, with_grad=False)
+    rows = [(0, h, r) for h in (0, 17) for r in (0, 5, k, 300, 511, 512, 1022, 1023)]
+    _check_fwd(x, "sparse", k, TOL_BF16, rows=rows)
+
+
+# --------------------------------------------------------------------- backward
+
+def _check_bwd(x, tol, heads=None):
+    d = _dev(x)
+    O, LSE = gb.forward(d["Q"], d["K"], d["V"], d["S"], mode="train")
+    dQ, dK, dV, dS = gb.backward(d["Q"], d["K"], d["V"], d["S"], O, LSE, d["dO"])
+    torch.cuda.synchronize()
+    ref = oracle.gated_attention_backward(np64(x["Q"]), np64(x["K"]), np64(x["V"]), x["S"].numpy(),
+                                          np64(x["dO"]), 64, heads=heads)
+    errs = {n: rel_err(np64(t) if t.dtype != torch.float32 else t.cpu().numpy().astype(np.float64), r)
+            for n, t, r in zip(("dQ", "dK", "dV", "dS"), (dQ, dK, dV, dS), ref[:4])}
+    for n, e in errs.items():
+        assert e < tol, (n, errs)
+    return errs
+
+
+def test_bwd_tiny_f32():
+    errs = _check_bwd(make_prefill_inputs(WORKLOADS["tiny_f32_n1024"]), TOL_GRAD)
+    assert max(errs.values()) < 1e-4, errs  # the fp32 path is far inside the bound
+
+
+@pytest.mark.parametrize("scaled", [True, False])
+def test_bwd_bf16_small(scaled):
+    _check_bwd(_small(5, 1, 8, 2, 1024, 128, torch.bfloat16, scaled), TOL_GRAD)
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 2, 64, 128), (2, 4, 4, 320, 64), (1, 4, 1, 448, 128)])
+def test_bwd_edge_shapes(shape):
+    B, Hq, Hkv, N, d = shape
+    for dtype in (torch.bfloat16, torch.float32):
+        _check_bwd(_small(3, B, Hq, Hkv, N, d, dtype, scaled=False), TOL_GRAD)
+
+
+def test_bwd_train_full_size_one_group():
+    """Training workload N=8192, 32/8 heads: all gradients of kv-group 0."""
+    w = WORKLOADS["train_bf16_n8192"]
+    _check_bwd(make_prefill_inputs(w), TOL_GRAD, heads=[(0, 0)])
+
+
+# ----------------------------------------------------------------------- decode
+
+def _check_decode(x, L, k, tol, seqs, num_splits=0):
+    O, LSE = gb.decode(x["q"].to(DEV), x["Kc"].to(DEV), x["Vc"].to(DEV), x["S"].to(DEV), L=L,
+                       topk=k, num_splits=num_splits)
+    torch.cuda.synchronize()
+    Kc = x["Kc"][seqs].cpu() if x["Kc"].is_cuda else x["Kc"][seqs]
+    Vc = x["Vc"][seqs].cpu() if x["Vc"].is_cuda else x["Vc"][seqs]
+    Or, Lr = oracle.gated_decode(np64(x["q"][seqs]), np64(Kc), np64(Vc), x["S"][seqs].cpu().numpy(),
+                                 L, 64, k)
+    eo = rel_err(np64(O[seqs]), Or)
+    el = rel_err(LSE[seqs].cpu().numpy(), Lr)
+    assert eo < tol and el < tol, (eo, el)
+
+
+@pytest.mark.parametrize("L", [64, 4096, 4133])
+@pytest.mark.parametrize("splits", [0, 1, 3])
+def test_decode_small(L, splits):
+    from dataclasses import replace
+    w = replace(WORKLOADS["sparse_decode_bf16_b64_l131072"], B=4, N=L)
+    x = make_decode_inputs(w, B=4, L=L)
+    _check_decode(x, L, 8, TOL_BF16, seqs=[0, 1, 2, 3], num_splits=splits)
+
+
+def test_decode_f32_small():
+    from dataclasses import replace
+    w = replace(WORKLOADS["sparse_decode_bf16_b64_l131072"], B=2, N=2000, dtype="f32")
+    x = make_decode_inputs(w, B=2, L=2000)
+    _check_decode(x, 2000, 5, TOL_F32, seqs=[0, 1])
+
+
+def test_decode_full_size_sampled():
+    """64 sequences x 131072 cache, K=32: sampled sequences against the oracle."""
+    w = WORKLOADS["sparse_decode_bf16_b64_l131072"]
+    x = make_decode_inputs(w, device=DEV)
+    _check_decode(x, w.N, 32, TOL_BF16, seqs=[0, 37, 63])
+    del x
+    torch.cuda.empty_cache()
