@@ -1,11 +1,512 @@
-// fwd_tc.cu — tensor-core (tcgen05) gated forward; placeholder until written.
+// fwd_tc.cu — K2: gated flash-attention forward on the 5th-generation tensor
+// cores (tcgen05, sm_100a), bf16 in, fp32 accumulate.
+//
+// Computes, per query row i, O_i = softmax_j(z_ij) V and LSE_i with
+// z_ij = scale * q_i.k_j + b_ij: b_ij is the normalised log gate of key block
+// c(j) for query block r(i) when c(j) is an attended historical block, 0 for
+// the current block with j <= i, -inf otherwise (ai.viyan.live, "SAS Learns
+// Token Importance for Sparse Attention", "The Logit Injection Mechanism";
+// Hugging Face paper page of "SAS: Simple Attention Sparsification via
+// End-to-End Optimization of Context Ranking", Abstract). Training mode visits
+// every block c <= r; sparse mode visits the Top-K list of K1 plus the current
+// block (NeurIPS 2026 poster page, Abstract). Blocks are processed one tile at
+// a time with an online softmax; the N x N matrix is never formed (blog,
+// "Implementation and Efficiency").
+//
+// Tiling: one CTA per (batch, q-head, 128-row query tile = two 64-row query
+// blocks). Each pipeline stage brings 128 keys = two 64-key "slots"; a slot is
+// one context block, so in sparse mode the two slots of a stage can be any two
+// blocks of the union of the tile's two selection lists (a per-tile "plan"
+// built by plan_kernel). Per slot and per query-block half the softmax applies
+// one scalar bias (log gate), a causal mask (current block) or -inf.
+//
+// Warp roles (192 threads): warps 0-3 softmax/epilogue (thread = query row =
+// TMEM lane), warp 4 TMA producer, warp 5 TMEM allocator + MMA issuer.
+// TMEM (512 columns): S double buffer at columns 0 and 128 (128 fp32 each),
+// O accumulator at 256. P is written back as bf16 over the first 64 columns
+// of its S buffer and consumed directly from TMEM by the PV MMA.
+// S = Q K^T: M=128, N=128, K=16 per instruction, both operands K-major,
+// 128-byte swizzled tiles loaded by TMA. O += P V: A = P from TMEM, B = V
+// MN-major (V rows are keys, contiguous in d).
+// The O rescale is lazy: the running max only moves when a row's new max
+// exceeds it by more than 2^8, which keeps the result exact (the final
+// normalisation uses the same max) while avoiding most TMEM round trips.
+// Every mbarrier wait is bounded; on expiry the kernel records
+// GBS_ERR_TIMEOUT, drains its MMAs and loads, frees TMEM and returns.
+#include <cuda.h>
+#include <stdio.h>
+
+#include "common.cuh"
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace gbs {
-bool fwd_tc_supported(const Problem&) { return false; }
-cudaError_t launch_fwd_tc(const Problem&, const void*, const void*, const void*, const float*,
-                          const Selection&, const int32_t*, int, void*, float*, unsigned int*,
-                          cudaStream_t) {
-  return cudaErrorNotSupported;
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 128;            // query rows per tile
+constexpr int kSlot = 64;           // keys per slot (one context block)
+constexpr int kBN = 2 * kSlot;      // keys per stage
+constexpr int kStages = 2;
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 512;
+constexpr uint64_t kTimeoutNs = 4000000000ull;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct Layout {
+  static constexpr int kChunks = D / 64;                   // 64-column (128-byte) chunks
+  static constexpr int kQChunk = kBM * 128;                // bytes per Q chunk
+  static constexpr int kKVChunk = kBN * 128;               // bytes per K/V chunk of a stage
+  static constexpr int kQBytes = kChunks * kQChunk;
+  static constexpr int kKVBytes = kChunks * kKVChunk;      // per stage, per tensor
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + kQBytes;
+  static constexpr int kVOff = kKOff + kStages * kKVBytes;
+  static constexpr int kBarOff = kVOff + kStages * kKVBytes;
+  static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers + alignment slack
+};
+
+struct Barriers {
+  uint64_t q_full;
+  uint64_t k_full[kStages];
+  uint64_t v_full[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_done;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct FwdArgs {
+  Problem p;
+  const float* S;
+  const float* slse;
+  const int32_t* plan;
+  int plan_stride;
+  int n_tiles;           // query tiles per head
+  __nv_bfloat16* O;
+  float* LSE;
+  unsigned int* err;
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
+
+// Slot `s` (0 or 1) of stage `j`: the key block to load.
+__device__ __forceinline__ int slot_block(const FwdArgs& a, const int32_t* plan_tile, int j, int s) {
+  if (a.p.mode == GBS_TRAIN) {
+    const int c = 2 * j + s;
+    return c < a.p.Nb ? c : 0;  // a block past the end (odd Nb) loads block 0, fully masked
+  }
+  return plan_tile[1 + 2 * j + s];
+}
+
+// Bias (log2 units) of slot `s` of stage `j` for query block `myr` of this
+// tile's half `half`: +inf marks the causal current block, -inf a masked slot.
+__device__ __forceinline__ float slot_bias(const FwdArgs& a, const int32_t* plan_tile, size_t bh,
+                                           int j, int s, int half, int myr) {
+  if (a.p.mode == GBS_TRAIN) {
+    const int c = 2 * j + s;
+    if (myr >= a.p.Nb || c > myr) return -INFINITY;
+    if (c == myr) return INFINITY;
+    const size_t row = bh * a.p.Nb + myr;
+    return (__ldg(a.S + row * a.p.Nb + c) - __ldg(a.slse + row)) * GBS_LOG2E;
+  }
+  return __int_as_float(__ldg(plan_tile + (1 + half) * a.plan_stride + 2 * j + s));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, FwdArgs a) {
+  using L = Layout<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  Barriers* bars = reinterpret_cast<Barriers*>(smem + L::kBarOff);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // heavy tiles first: consecutive CTAs are the heads of one tile (KV reuse in L2)
+  const int BH = a.p.B * a.p.Hq;
+  const int tile = a.n_tiles - 1 - (int)(blockIdx.x / BH);
+  const int bh = (int)(blockIdx.x % BH);
+  const int b = bh / a.p.Hq, h = bh % a.p.Hq;
+  const int kvz = b * a.p.Hkv + h / a.p.G;
+  const int32_t* plan_tile =
+      a.p.mode == GBS_TRAIN ? nullptr : a.plan + ((size_t)bh * a.n_tiles + tile) * 3 * a.plan_stride;
+  const int n_stages = a.p.mode == GBS_TRAIN ? tile + 1 : (__ldg(plan_tile) >> 1);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->s_full[s], 1);
+      mbar_init(&bars->p_full[s], 128);
+    }
+    mbar_init(&bars->o_done, 1);
+    mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  if (warp == 5) {
+    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  volatile int* abort_flag = &bars->abort_flag;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      constexpr uint32_t kSlotBytes = kSlot * 128;
+      mbar_arrive_expect_tx(&bars->q_full, L::kQBytes);
+      for (int ch = 0; ch < L::kChunks; ++ch)
+        tma_load_3d(smem + L::kQOff + ch * L::kQChunk, &tmQ, &bars->q_full, ch * 64, tile * kBM, bh);
+      int issued = 0;
+      for (int j = 0; j < n_stages; ++j) {
+        const int st = j % kStages;
+        if (j >= kStages &&
+            !mbar_wait(&bars->kv_empty[st], ((j / kStages) - 1) & 1, abort_flag, a.err, kTimeoutNs))
+          break;
+        const int c0 = slot_block(a, plan_tile, j, 0), c1 = slot_block(a, plan_tile, j, 1);
+        uint8_t* kst = smem + L::kKOff + st * L::kKVBytes;
+        uint8_t* vst = smem + L::kVOff + st * L::kKVBytes;
+        mbar_arrive_expect_tx(&bars->k_full[st], L::kKVBytes);
+        for (int ch = 0; ch < L::kChunks; ++ch) {
+          tma_load_3d(kst + ch * L::kKVChunk, &tmK, &bars->k_full[st], ch * 64, c0 * kSlot, kvz);
+          tma_load_3d(kst + ch * L::kKVChunk + kSlotBytes, &tmK, &bars->k_full[st], ch * 64,
+                      c1 * kSlot, kvz);
+        }
+        mbar_arrive_expect_tx(&bars->v_full[st], L::kKVBytes);
+        for (int ch = 0; ch < L::kChunks; ++ch) {
+          tma_load_3d(vst + ch * L::kKVChunk, &tmV, &bars->v_full[st], ch * 64, c0 * kSlot, kvz);
+          tma_load_3d(vst + ch * L::kKVChunk + kSlotBytes, &tmV, &bars->v_full[st], ch * 64,
+                      c1 * kSlot, kvz);
+        }
+        issued = j + 1;
+      }
+      if (*abort_flag) {
+        // let the loads still in flight land before the CTA exits
+        mbar_wait(&bars->q_full, 0, abort_flag, nullptr, 1000000ull);
+        for (int j = issued - kStages < 0 ? 0 : issued - kStages; j < issued; ++j) {
+          mbar_wait(&bars->k_full[j % kStages], (j / kStages) & 1, abort_flag, nullptr, 1000000ull);
+          mbar_wait(&bars->v_full[j % kStages], (j / kStages) & 1, abort_flag, nullptr, 1000000ull);
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // -------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(kBM, kBN, 0);
+      constexpr uint32_t idO = idesc_bf16_f32(kBM, D, 1);
+      const uint32_t q_addr = smem_u32(smem + L::kQOff);
+      const uint32_t tO = tmem + 256;
+      bool ok = mbar_wait(&bars->q_full, 0, abort_flag, a.err, kTimeoutNs);
+      auto issue_pv = [&](int i) -> bool {
+        const int st = i % kStages;
+        if (!mbar_wait(&bars->p_full[i & 1], (i >> 1) & 1, abort_flag, a.err, kTimeoutNs)) return false;
+        if (!mbar_wait(&bars->v_full[st], (i / kStages) & 1, abort_flag, a.err, kTimeoutNs)) return false;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(smem + L::kVOff + st * L::kKVBytes);
+        const uint32_t tP = tmem + (i & 1) * 128;
+#pragma unroll
+        for (int ks = 0; ks < kBN / 16; ++ks) {
+          const uint64_t bdesc = sdesc_sw128(v_addr + ks * 16 * 128, L::kKVChunk, 1024);
+          mma_ts(tO, tP + ks * 8, bdesc, idO, (i > 0 || ks > 0) ? 1u : 0u);
+        }
+        mma_commit(&bars->o_done);
+        mma_commit(&bars->kv_empty[st]);
+        return true;
+      };
+      for (int j = 0; ok && j < n_stages; ++j) {
+        const int st = j % kStages;
+        if (!mbar_wait(&bars->k_full[st], (j / kStages) & 1, abort_flag, a.err, kTimeoutNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(smem + L::kKOff + st * L::kKVBytes);
+        const uint32_t tS = tmem + (j & 1) * 128;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const int ch = ks >> 2, kk = ks & 3;
+          const uint64_t adesc = sdesc_sw128(q_addr + ch * L::kQChunk + kk * 32, 16, 1024);
+          const uint64_t bdesc = sdesc_sw128(k_addr + ch * L::kKVChunk + kk * 32, 16, 1024);
+          mma_ss(tS, adesc, bdesc, idS, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars->s_full[j & 1]);
+        if (j > 0 && !issue_pv(j - 1)) ok = false;
+      }
+      if (ok) issue_pv(n_stages - 1);
+      // drain: every MMA issued above has finished once this arrives
+      mma_commit(&bars->drain);
+      mbar_wait(&bars->drain, 0, abort_flag, a.err, kTimeoutNs);
+    }
+  } else {
+    // ----------------------------------------------------- softmax + epilogue
+    const int row = warp * 32 + lane;  // TMEM lane == query row in the tile
+    const int half = row >> 6, iloc = row & 63;
+    const int myr = 2 * tile + half;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const float sc = a.p.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_stages; ++j) {
+      const float bias0 = slot_bias(a, plan_tile, bh, j, 0, half, myr);
+      const float bias1 = slot_bias(a, plan_tile, bh, j, 1, half, myr);
+      if (!mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1, abort_flag, a.err, kTimeoutNs)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tS = tmem + lane_off + (j & 1) * 128;
+      uint32_t raw[4][32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, raw[q]);
+      tmem_wait_ld();
+      float v[128];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < 128; ++k) {
+        const float bias = k < 64 ? bias0 : bias1;
+        const int kl = k & 63;
+        float x = __uint_as_float(raw[k >> 5][k & 31]);
+        if (bias == INFINITY)
+          x = kl <= iloc ? x * sc : -INFINITY;
+        else
+          x = bias == -INFINITY ? -INFINITY : fmaf(x, sc, bias);
+        v[k] = x;
+        mx = fmaxf(mx, x);
+      }
+      const bool need = mx > m + kRescaleThreshold;
+      // PV of the previous stage must be complete before O is touched; waiting
+      // every stage also keeps the o_done parity unambiguous.
+      if (j > 0) {
+        if (!mbar_wait(&bars->o_done, (j - 1) & 1, abort_flag, a.err, kTimeoutNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, need) && j > 0) {
+        const float f = need ? ex2(m - mx) : 1.f;
+        const uint32_t tO = tmem + lane_off + 256;
+#pragma unroll
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t o[32];
+          tmem_ld32(tO + q * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
+          tmem_st32(tO + q * 32, o);
+        }
+        l *= f;
+      }
+      if (need) m = mx;
+      const float mu = m == -INFINITY ? 0.f : m;
+      uint32_t pk[2][32];
+      float ls = 0.f;
+#pragma unroll
+      for (int k = 0; k < 64; ++k) {
+        const float p0 = ex2(v[2 * k] - mu), p1 = ex2(v[2 * k + 1] - mu);
+        ls += p0 + p1;
+        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+        pk[k >> 5][k & 31] = *reinterpret_cast<const uint32_t*>(&pb);
+      }
+      l += ls;
+      tmem_st32(tS, pk[0]);
+      tmem_st32(tS + 32, pk[1]);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[j & 1]);
+    }
+    if (ok && mbar_wait(&bars->o_done, (n_stages - 1) & 1, abort_flag, a.err, kTimeoutNs)) {
+      tc_fence_after();
+      const int qrow = tile * kBM + row;
+      const bool valid = qrow < a.p.N;
+      const float inv = 1.f / l;
+      const uint32_t tO = tmem + lane_off + 256;
+      __nv_bfloat16* orow = a.O + ((size_t)bh * a.p.N + qrow) * D;
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t o[32];
+        tmem_ld32(tO + q * 32, o);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(o[2 * k]) * inv,
+                                                          __uint_as_float(o[2 * k + 1]) * inv);
+          pk[k] = *reinterpret_cast<const uint32_t*>(&pb);
+        }
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) dst[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+        }
+      }
+      if (valid) a.LSE[(size_t)bh * a.p.N + qrow] = (m + log2f(l)) * GBS_LN2;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Per (batch, head, tile): the ascending union of both query blocks' selected
+// lists plus their current blocks, padded to an even slot count, with each
+// half's bias per slot (log2 units; +inf = causal current block, -inf = not
+// attended by that half).
+__global__ void plan_kernel(Problem p, Selection sel, int32_t* __restrict__ plan, int stride,
+                            int n_tiles) {
+  const int id = blockIdx.x * blockDim.x + threadIdx.x;
+  const int BH = p.B * p.Hq;
+  if (id >= BH * n_tiles) return;
+  const int bh = id / n_tiles, t = id % n_tiles;
+  int32_t* out = plan + (size_t)id * 3 * stride;
+  int32_t* cs = out + 1;
+  float* b0 = reinterpret_cast<float*>(out + stride);
+  float* b1 = reinterpret_cast<float*>(out + 2 * stride);
+  const int r0 = 2 * t, r1 = 2 * t + 1;
+  const bool has1 = r1 < p.Nb;
+  const size_t row0 = (size_t)bh * p.Nb + r0, row1 = row0 + 1;
+  const int n0 = sel.cnt[row0], n1 = has1 ? sel.cnt[row1] : 0;
+  const int32_t* i0 = sel.idx + row0 * p.topk;
+  const int32_t* i1 = sel.idx + row1 * p.topk;
+  const float* g0 = sel.logg + row0 * p.topk;
+  const float* g1 = sel.logg + row1 * p.topk;
+  int a0 = 0, a1 = 0, n = 0;
+  bool d0 = false, d1 = !has1;
+  while (true) {
+    // next candidate block from each source (INT_MAX when exhausted)
+    const int x0 = a0 < n0 ? i0[a0] : 0x7fffffff;
+    const int x1 = a1 < n1 ? i1[a1] : 0x7fffffff;
+    const int xd0 = d0 ? 0x7fffffff : r0;
+    const int xd1 = d1 ? 0x7fffffff : r1;
+    const int c = min(min(x0, x1), min(xd0, xd1));
+    if (c == 0x7fffffff) break;
+    float v0 = -INFINITY, v1 = -INFINITY;
+    if (x0 == c) { v0 = g0[a0++] * GBS_LOG2E; }
+    if (xd0 == c) { v0 = INFINITY; d0 = true; }
+    if (x1 == c) { v1 = g1[a1++] * GBS_LOG2E; }
+    if (xd1 == c) { v1 = INFINITY; d1 = true; }
+    cs[n] = c;
+    b0[n] = v0;
+    b1[n] = v1;
+    ++n;
+  }
+  if (n & 1) {  // pad: reload the last block, attended by nobody
+    cs[n] = cs[n - 1];
+    b0[n] = -INFINITY;
+    b1[n] = -INFINITY;
+    ++n;
+  }
+  out[0] = n;
+}
+
+// --------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// [rows_per_head, d] bf16 per head, heads stacked: dims (d, rows, heads).
+bool make_map(CUtensorMap* m, const void* base, int d, int rows, int heads, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)heads};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * rows * 2};
+  const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_typed(const FwdArgs& a, const void* Q, const void* K, const void* V,
+                         cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, Q, D, a.p.N, a.p.B * a.p.Hq, kBM) ||
+      !make_map(&tk, K, D, a.p.N, a.p.B * a.p.Hkv, kSlot) ||
+      !make_map(&tv, V, D, a.p.N, a.p.B * a.p.Hkv, kSlot))
+    return cudaErrorInvalidValue;
+  auto kern = fwd_tc_kernel<D>;
+  const int smem = Layout<D>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)(a.p.B * a.p.Hq * a.n_tiles);
+  kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool fwd_tc_supported(const Problem& p) {
+  return p.dtype == GBS_BF16 && p.bs == kSlot && (p.d == 64 || p.d == 128) && p.N % kSlot == 0;
+}
+
+cudaError_t launch_fwd_tc(const Problem& p, const void* Q, const void* K, const void* V,
+                          const float* S, const Selection& sel, const int32_t* plan,
+                          int plan_stride, void* O, float* LSE, unsigned int* err,
+                          cudaStream_t st) {
+  if (!fwd_tc_supported(p)) return cudaErrorNotSupported;
+  FwdArgs a;
+  a.p = p;
+  a.S = S;
+  a.slse = sel.slse;
+  a.plan = plan;
+  a.plan_stride = plan_stride;
+  a.n_tiles = (p.Nb + 1) / 2;
+  a.O = reinterpret_cast<__nv_bfloat16*>(O);
+  a.LSE = LSE;
+  a.err = err;
+  if (p.mode == GBS_SPARSE) {
+    const int n = p.B * p.Hq * a.n_tiles;
+    plan_kernel<<<(n + 127) / 128, 128, 0, st>>>(p, sel, const_cast<int32_t*>(plan), plan_stride,
+                                                 a.n_tiles);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (p.d == 64) return launch_typed<64>(a, Q, K, V, st);
+  return launch_typed<128>(a, Q, K, V, st);
+}
+
 }  // namespace gbs
