@@ -22,7 +22,8 @@ DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 OP_FWD, OP_BWD, OP_DECODE = 0, 1, 2
 
 EXPORTED = ("gbs_version", "gbs_status_string", "gbs_last_error", "gbs_workspace_bytes",
-            "gbs_clear_error", "gbs_check", "gbs_select", "gbs_fwd", "gbs_bwd", "gbs_decode")
+            "gbs_clear_error", "gbs_check", "gbs_select", "gbs_fwd", "gbs_bwd", "gbs_decode",
+            "gbs_set_timer", "gbs_launch_count")
 
 
 class GbsError(RuntimeError):
@@ -62,6 +63,8 @@ def load_library(path: str = LIB_PATH):
         "gbs_fwd": (i32, [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "gbs_bwd": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "gbs_decode": (i32, [P, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]),
+        "gbs_set_timer": (i32, [i32, vp, vp]),
+        "gbs_launch_count": (ctypes.c_uint64, []),
     }
     for name, (res, args) in sigs.items():
         f = getattr(lib, name)
@@ -169,6 +172,22 @@ def decode(q, Kc, Vc, S, L=None, block=64, topk=32, scale=0.0, num_splits=0, out
     _check(lib.gbs_decode(ctypes.byref(p), _ptr(q), _ptr(Kc), _ptr(Vc), _ptr(S), _ptr(O), _ptr(LSE),
                           num_splits, _ptr(ws), ws.numel(), _stream(stream)), "gbs_decode")
     return O, LSE
+
+
+def set_timer(op: int, start=None, stop=None):
+    """Brackets the main kernel of ``op`` with two recorded torch.cuda.Events.
+
+    The events must already exist on the device (record them once first).
+    Pass None to clear.
+    """
+    h0 = None if start is None else ctypes.c_void_p(start.cuda_event)
+    h1 = None if stop is None else ctypes.c_void_p(stop.cuda_event)
+    _check(load_library().gbs_set_timer(op, h0, h1), "gbs_set_timer")
+
+
+def launch_count() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(load_library().gbs_launch_count())
 
 
 def check(ws, stream=None):

@@ -275,6 +275,7 @@ cudaError_t fwd_simt_typed(const Problem& p, const void* Q, const void* K, const
   if (e != cudaSuccess) return e;
   dim3 grid(p.Nb, p.Hq, p.B);
   kern<<<grid, kBS, smem, st>>>(p, (const T*)Q, (const T*)K, (const T*)V, S, sel, (T*)O, LSE);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -286,6 +287,7 @@ cudaError_t bwd_simt_typed(const Problem& p, const void* Q, const void* K, const
   const size_t rows = (size_t)p.B * p.Hq * p.N;
   bwd_dot_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>((const T*)O, (const T*)dO,
                                                                    Dvec, rows);
+  note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   {
@@ -293,8 +295,10 @@ cudaError_t bwd_simt_typed(const Problem& p, const void* Q, const void* K, const
     auto kern = bwd_dq_kernel<T, D>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    timer_begin(GBS_OP_BWD, st);
     kern<<<dim3(p.Nb, p.Hq, p.B), kBS, smem, st>>>(p, (const T*)Q, (const T*)K, (const T*)V, S,
                                                     slse, LSE, (const T*)dO, Dvec, (T*)dQ, Gblk);
+    note_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   {
@@ -305,10 +309,13 @@ cudaError_t bwd_simt_typed(const Problem& p, const void* Q, const void* K, const
     kern<<<dim3(p.Nb, p.Hkv, p.B), 2 * kBS, smem, st>>>(p, (const T*)Q, (const T*)K, (const T*)V,
                                                          S, slse, LSE, (const T*)dO, Dvec,
                                                          (T*)dK, (T*)dV);
+    note_launch();
+    timer_end(GBS_OP_BWD, st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   const size_t srows = (size_t)p.B * p.Hq * p.Nb;
   ds_finalize_kernel<<<(unsigned)((srows + 7) / 8), 256, 0, st>>>(S, slse, Gblk, dS, p.Nb, srows);
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -196,11 +196,15 @@ cudaError_t decode_typed(const Problem& p, const void* q, const void* Kc, const 
                          const Selection& sel, int cur, int splits, float* part_ml,
                          float* part_acc, void* O, float* LSE, cudaStream_t st) {
   const int BH = p.B * p.Hq;
+  timer_begin(GBS_OP_DECODE, st);
   decode_split_kernel<T, D><<<dim3(BH, splits), kThreads, 0, st>>>(
       p, (const T*)q, (const T*)Kc, (const T*)Vc, sel, cur, splits, part_ml, part_acc);
+  timer_end(GBS_OP_DECODE, st);
+  note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_combine_kernel<T, D><<<BH, D, 0, st>>>(p, splits, part_ml, part_acc, (T*)O, LSE);
+  note_launch();
   return cudaGetLastError();
 }
 

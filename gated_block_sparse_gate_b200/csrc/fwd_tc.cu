@@ -473,7 +473,10 @@ cudaError_t launch_typed(const FwdArgs& a, const void* Q, const void* K, const v
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)(a.p.B * a.p.Hq * a.n_tiles);
+  timer_begin(GBS_OP_FWD, st);
   kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, a);
+  timer_end(GBS_OP_FWD, st);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -502,6 +505,7 @@ cudaError_t launch_fwd_tc(const Problem& p, const void* Q, const void* K, const 
     const int n = p.B * p.Hq * a.n_tiles;
     plan_kernel<<<(n + 127) / 128, 128, 0, st>>>(p, sel, const_cast<int32_t*>(plan), plan_stride,
                                                  a.n_tiles);
+    note_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -1,6 +1,7 @@
 // gbs_api.cu — the C ABI declared in include/gbs.h: argument validation,
 // workspace layout and kernel dispatch. No allocation, no synchronisation
 // (except gbs_check), no host-side compute.
+#include <atomic>
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
@@ -12,6 +13,9 @@
 using namespace gbs;
 
 namespace {
+
+std::atomic<unsigned long long> g_launches{0};
+cudaEvent_t g_timer[3][2] = {};
 
 thread_local char g_last_error[256] = "";
 
@@ -155,7 +159,29 @@ unsigned int* err_word(void* ws) { return reinterpret_cast<unsigned int*>(ws); }
 
 }  // namespace
 
+namespace gbs {
+void note_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+void timer_begin(int op, cudaStream_t st) {
+  if (g_timer[op][0]) cudaEventRecord(g_timer[op][0], st);
+}
+void timer_end(int op, cudaStream_t st) {
+  if (g_timer[op][1]) cudaEventRecord(g_timer[op][1], st);
+}
+}  // namespace gbs
+
 extern "C" {
+
+gbs_status gbs_set_timer(int op, void* start, void* stop) {
+  if (op < GBS_OP_FWD || op > GBS_OP_DECODE) return fail(GBS_ERR_INVALID_ARG, "op %d unknown", op);
+  if ((start == nullptr) != (stop == nullptr))
+    return fail(GBS_ERR_INVALID_ARG, "set both timer events or neither");
+  g_timer[op][0] = (cudaEvent_t)start;
+  g_timer[op][1] = (cudaEvent_t)stop;
+  return GBS_OK;
+}
+
+uint64_t gbs_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
 
 int gbs_version(void) { return (GBS_VERSION_MAJOR << 16) | GBS_VERSION_MINOR; }
 
@@ -236,7 +262,10 @@ gbs_status gbs_fwd(const gbs_params* in, const void* Q, const void* K, const voi
     e = launch_fwd_tc(p, Q, K, V, S, w.sel, w.plan, (int)plan_stride(p), O, LSE, err_word(ws), st);
     if (e != cudaErrorNotSupported) return cuda_status(e, "gbs_fwd/attention");
   }
-  return cuda_status(launch_fwd_simt(p, Q, K, V, S, w.sel, O, LSE, st), "gbs_fwd/attention");
+  timer_begin(GBS_OP_FWD, st);
+  e = launch_fwd_simt(p, Q, K, V, S, w.sel, O, LSE, st);
+  timer_end(GBS_OP_FWD, st);
+  return cuda_status(e, "gbs_fwd/attention");
 }
 
 gbs_status gbs_bwd(const gbs_params* in, const void* Q, const void* K, const void* V,

@@ -9,6 +9,12 @@
 
 namespace gbs {
 
+// Bookkeeping shared by all launchers: every kernel launch is counted, and
+// the main kernel of an op is bracketed by the caller's timer events if set.
+void note_launch(int n = 1);
+void timer_begin(int op, cudaStream_t st);
+void timer_end(int op, cudaStream_t st);
+
 // Resolved problem description handed to every launcher.
 struct Problem {
   int B, Hq, Hkv, N, d, bs, Nb, G, topk, mode, dtype;

@@ -127,6 +127,7 @@ cudaError_t launch_select(const float* S, int n_rows, int row_stride, int rows_p
   const int grid = (n_rows + kWarps - 1) / kWarps;
   select_kernel<<<grid, kWarps * 32, 0, st>>>(S, n_rows, row_stride, rows_per_head, decode_cur,
                                               topk, sparse ? 1 : 0, idx, cnt, logg, slse);
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -157,6 +157,17 @@ GBS_API gbs_status gbs_decode(const gbs_params* p, const void* q, const void* Kc
                       const float* S, void* O, float* LSE, int num_splits, void* ws,
                       size_t ws_bytes, void* stream);
 
+/* Profiling hook: while `start`/`stop` (cudaEvent_t, caller-owned) are set for
+ * `op`, every call of that op records `start` on its stream immediately before
+ * its main attention kernel and `stop` immediately after it, so the caller can
+ * time that one kernel. Pass NULL to clear. Process-wide, not thread-safe; the
+ * main kernel is the tensor-core (or SIMT) attention kernel for GBS_OP_FWD and
+ * GBS_OP_BWD and the split kernel for GBS_OP_DECODE. */
+GBS_API gbs_status gbs_set_timer(int op, void* start, void* stop);
+
+/* Total number of CUDA kernels this library has launched in this process. */
+GBS_API uint64_t gbs_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif
