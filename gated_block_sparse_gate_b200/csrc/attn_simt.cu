@@ -321,6 +321,14 @@ cudaError_t bwd_simt_typed(const Problem& p, const void* Q, const void* K, const
 
 }  // namespace
 
+cudaError_t launch_ds_finalize(const Problem& p, const float* S, const float* slse,
+                               const float* Gblk, float* dS, cudaStream_t st) {
+  const size_t srows = (size_t)p.B * p.Hq * p.Nb;
+  ds_finalize_kernel<<<(unsigned)((srows + 7) / 8), 256, 0, st>>>(S, slse, Gblk, dS, p.Nb, srows);
+  note_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_fwd_simt(const Problem& p, const void* Q, const void* K, const void* V,
                             const float* S, const Selection& sel, void* O, float* LSE,
                             cudaStream_t st) {

@@ -1,0 +1,530 @@
+// bwd_tc.cu — K3: gated attention backward (training mode) on the tcgen05
+// tensor cores, with the tile sums G that give dS fused in.
+//
+// The gradient flows from the loss through the softmax into the selector
+// scores because the gate sits inside the softmax in log form (ai.viyan.live,
+// "SAS Learns Token Importance for Sparse Attention", "The Logit Injection
+// Mechanism"; NeurIPS 2026 poster page of "SAS: Simple Attention
+// Sparsification via End-to-End Optimization of Context Ranking", Abstract:
+// every context unit stays active in training so each one receives gradient).
+// With P = exp(z - LSE), dP = dO V^T, dZ = P o (dP - D), D_i = dO_i . O_i:
+//   dV = P^T dO, dK = scale dZ^T Q, dQ = scale dZ K,
+//   G[r, c] = sum of dZ over the (query block r, key block c) tile.
+// dS[r, c'] = G[r, c'] - g[r, c'] sum_{c<r} G[r, c] is formed afterwards from G.
+//
+// Tiling: one CTA per (batch, kv-head, 128-key tile = two 64-key context
+// blocks); K and V stay in shared memory while the CTA walks the G q-heads of
+// the group and every 128-query tile at or after its keys. Per step:
+//   S^T = K Q^T and dP^T = V dO^T   (M=128 keys, N=128 queries, K=d; TMEM)
+//   compute warps: P^T, dZ^T (bf16) back into TMEM, dZ^T into swizzled smem,
+//                  per-warp sums of dZ added into G
+//   dV += P^T dO, dK += dZ^T Q      (A from TMEM, B = dO / Q MN-major)
+//   dQ  = dZ K                      (A = dZ^T smem MN-major, B = K MN-major;
+//                                    TMEM, drained by vector reductions into
+//                                    an fp32 accumulator in the workspace)
+// TMEM (512 columns): R0 = S^T / P^T / dQ, R1 = dP^T / dZ^T, dV, dK. The bf16
+// P^T and dZ^T of query half h are stored over the first 32 columns of that
+// half's own 64 S^T / dP^T columns.
+// Warps: 0-7 compute (lane quadrant w%4, query/column half w/4), 8 TMA,
+// 9 TMEM allocator + MMA issuer. Every mbarrier wait is bounded.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace gbs {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kBK = 128;         // keys per CTA
+constexpr int kBQ = 128;         // queries per step
+constexpr int kQStages = 2;
+constexpr int kComputeWarps = 8;
+constexpr int kThreads = (kComputeWarps + 2) * 32;
+constexpr int kTmemCols = 512;
+constexpr uint64_t kTimeoutNs = 4000000000ull;
+constexpr int kChunk = 128 * 128;  // bytes of one 64-column chunk of a 128-row tile
+
+template <int D>
+struct BLayout {
+  static constexpr int kChunks = D / 64;
+  static constexpr int kTile = kChunks * kChunk;  // one 128 x D bf16 tile
+  static constexpr int kKOff = 0;
+  static constexpr int kVOff = kKOff + kTile;
+  static constexpr int kQOff = kVOff + kTile;
+  static constexpr int kdOOff = kQOff + kQStages * kTile;
+  static constexpr int kZOff = kdOOff + kQStages * kTile;   // dZ^T: 128 keys x 128 queries
+  static constexpr int kVecOff = kZOff + 2 * kChunk;        // (lse2, D) per query, per stage
+  static constexpr int kBarOff = kVecOff + kQStages * kBQ * 8;
+  static constexpr int kSmemBytes = kBarOff + 256;
+};
+
+struct BBarriers {
+  uint64_t kv_full;
+  uint64_t q_full[kQStages];
+  uint64_t q_empty[kQStages];
+  uint64_t st_full;
+  uint64_t p_full;
+  uint64_t dq_full;
+  uint64_t dq_free;
+  uint64_t done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct BwdArgs {
+  Problem p;
+  const float* S;
+  const float* slse;
+  const float* LSE;
+  const float* Dvec;
+  float* dQacc;
+  float* Gblk;
+  __nv_bfloat16* dK;
+  __nv_bfloat16* dV;
+  int n_tiles;  // 128-row tiles per head (keys and queries alike)
+  unsigned int* err;
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+enum : int { kMasked = 0, kCausal = 1, kFull = 2 };
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+              BwdArgs a) {
+  using L = BLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {  // the swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) set_error(a.err, GBS_ERR_UNSUPPORTED);
+    return;
+  }
+  BBarriers* bars = reinterpret_cast<BBarriers*>(smem + L::kBarOff);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Problem& p = a.p;
+
+  const int BKV = p.B * p.Hkv;
+  const int u = (int)(blockIdx.x / BKV);  // key tile; small u = most work, launched first
+  const int bk = (int)(blockIdx.x % BKV);
+  const int b = bk / p.Hkv, kvh = bk % p.Hkv;
+  const int per_head = a.n_tiles - u;
+  const int n_steps = p.G * per_head;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->kv_full, 1);
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(&bars->q_full[s], 1);
+      mbar_init(&bars->q_empty[s], 1);
+    }
+    mbar_init(&bars->st_full, 1);
+    mbar_init(&bars->p_full, kComputeWarps * 32);
+    mbar_init(&bars->dq_full, 1);
+    mbar_init(&bars->dq_free, kComputeWarps * 32);
+    mbar_init(&bars->done, 1);
+    bars->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  volatile int* abort_flag = &bars->abort_flag;
+  float2* vecs = reinterpret_cast<float2*>(smem + L::kVecOff);
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      prefetch_tmap(&tmdO);
+      mbar_arrive_expect_tx(&bars->kv_full, 2 * L::kTile);
+      for (int ch = 0; ch < L::kChunks; ++ch) {
+        tma_load_3d(smem + L::kKOff + ch * kChunk, &tmK, &bars->kv_full, ch * 64, u * kBK, bk);
+        tma_load_3d(smem + L::kVOff + ch * kChunk, &tmV, &bars->kv_full, ch * 64, u * kBK, bk);
+      }
+    }
+    int issued = 0;
+    for (int j = 0; j < n_steps; ++j) {
+      const int st = j % kQStages;
+      int ok = 1;
+      if (lane == 0 && j >= kQStages)
+        ok = mbar_wait(&bars->q_empty[st], ((j / kQStages) - 1) & 1, abort_flag, a.err, kTimeoutNs);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      const int hh = j / per_head, t = u + j % per_head;
+      const int bh = b * p.Hq + kvh * p.G + hh;
+      const int q0 = t * kBQ;
+      float2* vec = vecs + st * kBQ;
+      for (int i = lane; i < kBQ; i += 32) {
+        const int q = q0 + i;
+        float2 v = make_float2(INFINITY, 0.f);  // rows past the end contribute nothing
+        if (q < p.N) {
+          const size_t idx = (size_t)bh * p.N + q;
+          v = make_float2(__ldg(a.LSE + idx) * GBS_LOG2E, __ldg(a.Dvec + idx));
+        }
+        vec[i] = v;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bars->q_full[st], 2 * L::kTile);
+        uint8_t* qs = smem + L::kQOff + st * L::kTile;
+        uint8_t* ds = smem + L::kdOOff + st * L::kTile;
+        for (int ch = 0; ch < L::kChunks; ++ch) {
+          tma_load_3d(qs + ch * kChunk, &tmQ, &bars->q_full[st], ch * 64, q0, bh);
+          tma_load_3d(ds + ch * kChunk, &tmdO, &bars->q_full[st], ch * 64, q0, bh);
+        }
+      }
+      issued = j + 1;
+    }
+    if (lane == 0 && *abort_flag) {
+      // let loads still in flight land before the CTA exits
+      mbar_wait(&bars->kv_full, 0, abort_flag, nullptr, 1000000ull);
+      for (int j = issued - kQStages < 0 ? 0 : issued - kQStages; j < issued; ++j)
+        mbar_wait(&bars->q_full[j % kQStages], (j / kQStages) & 1, abort_flag, nullptr, 1000000ull);
+    }
+  } else if (warp == 9) {
+    // -------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idST = idesc_bf16_f32(kBK, kBQ, 0, 0);  // S^T, dP^T
+      constexpr uint32_t idKV = idesc_bf16_f32(kBK, D, 1, 0);    // dV, dK (A in TMEM)
+      constexpr uint32_t idQ = idesc_bf16_f32(kBQ, D, 1, 1);     // dQ (A, B MN-major)
+      const uint32_t R0 = tmem, R1 = tmem + 128, TdV = tmem + 256, TdK = tmem + 384;
+      const uint32_t k_addr = smem_u32(smem + L::kKOff), v_addr = smem_u32(smem + L::kVOff);
+      const uint32_t z_addr = smem_u32(smem + L::kZOff);
+      bool ok = mbar_wait(&bars->kv_full, 0, abort_flag, a.err, kTimeoutNs);
+      auto issue_dp = [&](int j) -> bool {
+        const int st = j % kQStages;
+        if (!mbar_wait(&bars->q_full[st], (j / kQStages) & 1, abort_flag, a.err, kTimeoutNs))
+          return false;
+        tc_fence_after();
+        const uint32_t do_addr = smem_u32(smem + L::kdOOff + st * L::kTile);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const int ch = ks >> 2, kk = ks & 3;
+          mma_ss(R1, sdesc_sw128(v_addr + ch * kChunk + kk * 32, 16, 1024),
+                 sdesc_sw128(do_addr + ch * kChunk + kk * 32, 16, 1024), idST, ks > 0 ? 1u : 0u);
+        }
+        return true;
+      };
+      if (ok) ok = issue_dp(0);
+      for (int j = 0; ok && j < n_steps; ++j) {
+        const int st = j % kQStages;
+        const uint32_t q_addr = smem_u32(smem + L::kQOff + st * L::kTile);
+        const uint32_t do_addr = smem_u32(smem + L::kdOOff + st * L::kTile);
+        if (j > 0) {
+          if (!mbar_wait(&bars->dq_free, (j - 1) & 1, abort_flag, a.err, kTimeoutNs)) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const int ch = ks >> 2, kk = ks & 3;
+          mma_ss(R0, sdesc_sw128(k_addr + ch * kChunk + kk * 32, 16, 1024),
+                 sdesc_sw128(q_addr + ch * kChunk + kk * 32, 16, 1024), idST, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars->st_full);
+        if (!mbar_wait(&bars->p_full, j & 1, abort_flag, a.err, kTimeoutNs)) break;
+        tc_fence_after();
+        // P^T / dZ^T of query half hq sit in columns [64 hq, 64 hq + 32) of R0 / R1
+#pragma unroll
+        for (int ks = 0; ks < kBQ / 16; ++ks) {
+          const uint32_t acc = (j > 0 || ks > 0) ? 1u : 0u;
+          const uint32_t acol = (ks >> 2) * 64 + (ks & 3) * 8;
+          mma_ts(TdV, R0 + acol, sdesc_sw128(do_addr + ks * 2048, kChunk, 1024), idKV, acc);
+          mma_ts(TdK, R1 + acol, sdesc_sw128(q_addr + ks * 2048, kChunk, 1024), idKV, acc);
+        }
+#pragma unroll
+        for (int ks = 0; ks < kBK / 16; ++ks)
+          mma_ss(R0, sdesc_sw128(z_addr + ks * 2048, kChunk, 1024),
+                 sdesc_sw128(k_addr + ks * 2048, kChunk, 1024), idQ, ks > 0 ? 1u : 0u);
+        mma_commit(&bars->dq_full);
+        mma_commit(&bars->q_empty[st]);
+        if (j + 1 < n_steps && !issue_dp(j + 1)) break;
+      }
+      mma_commit(&bars->done);
+      mbar_wait(&bars->done, 0, abort_flag, a.err, kTimeoutNs);
+    }
+  } else {
+    // ------------------------------------------------------- compute warps
+    const int quad = warp & 3, hq = warp >> 2;
+    const int krow = quad * 32 + lane;  // key row within the tile == TMEM lane
+    const int cj = 2 * u + (krow >> 6), jloc = krow & 63;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const float sc = p.scale_log2;
+    uint8_t* zrow = smem + L::kZOff + hq * kChunk + krow * 128;
+    bool ok = true;
+    for (int j = 0; j < n_steps; ++j) {
+      const int st = j % kQStages;
+      const int hh = j / per_head, t = u + j % per_head;
+      const int bh = b * p.Hq + kvh * p.G + hh;
+      const int r = 2 * t + hq;  // this warp's query block
+      int mode = kFull;
+      float bias2 = 0.f;
+      if (r >= p.Nb || cj > r) {
+        mode = kMasked;
+      } else if (cj == r) {
+        mode = kCausal;
+      } else {
+        const size_t row = (size_t)bh * p.Nb + r;
+        bias2 = (__ldg(a.S + row * p.Nb + cj) - __ldg(a.slse + row)) * GBS_LOG2E;
+      }
+      if (!mbar_wait(&bars->st_full, j & 1, abort_flag, a.err, kTimeoutNs) ||
+          !mbar_wait(&bars->q_full[st], (j / kQStages) & 1, abort_flag, a.err, kTimeoutNs)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float2* vec = vecs + st * kBQ + hq * 64;
+      float g = 0.f;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {  // two chunks of 32 query columns
+        const uint32_t col = hq * 64 + c * 32;
+        uint32_t sv[32], dv[32], pp[16], zz[16];
+        tmem_ld32(tmem + lane_off + col, sv);
+        tmem_ld32(tmem + 128 + lane_off + col, dv);
+        tmem_wait_ld();
+        if (mode == kMasked) {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) pp[k] = zz[k] = 0u;
+        } else {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            float pr[2], dz[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int i = 2 * k + e;
+              const float2 ld = vec[c * 32 + i];
+              float x = fmaf(__uint_as_float(sv[i]), sc, bias2 - ld.x);
+              if (mode == kCausal && c * 32 + i < jloc) x = -INFINITY;
+              pr[e] = ex2(x);
+              dz[e] = pr[e] * (__uint_as_float(dv[i]) - ld.y);
+            }
+            g += dz[0] + dz[1];
+            pp[k] = pack_bf16(pr[0], pr[1]);
+            zz[k] = pack_bf16(dz[0], dz[1]);
+          }
+        }
+        // packed outputs stay inside this warp's own 64 columns of S^T / dP^T
+        // (which the other warp of the quadrant never reads), over columns
+        // already consumed by this chunk
+        tmem_st16(tmem + lane_off + hq * 64 + c * 16, pp);
+        tmem_st16(tmem + 128 + lane_off + hq * 64 + c * 16, zz);
+#pragma unroll
+        for (int gi = 0; gi < 4; ++gi) {
+          const int gg = c * 4 + gi;
+          *reinterpret_cast<uint4*>(zrow + ((gg ^ (krow & 7)) << 4)) =
+              make_uint4(zz[4 * gi], zz[4 * gi + 1], zz[4 * gi + 2], zz[4 * gi + 3]);
+        }
+      }
+      g = warp_sum(g);
+      if (lane == 0 && mode != kMasked) atomicAdd(a.Gblk + ((size_t)bh * p.Nb + r) * p.Nb + cj, g);
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full);
+
+      // drain dQ (TMEM lane == query row) into the fp32 accumulator
+      if (!mbar_wait(&bars->dq_full, j & 1, abort_flag, a.err, kTimeoutNs)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int qrow = t * kBQ + krow;
+      float* dst = a.dQacc + ((size_t)bh * p.N + qrow) * D + hq * (D / 2);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_off + hq * (D / 2) + c * 32, o);
+        tmem_wait_ld();
+        if (qrow < p.N) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            red_add_v4(dst + c * 32 + 4 * k, __uint_as_float(o[4 * k]), __uint_as_float(o[4 * k + 1]),
+                       __uint_as_float(o[4 * k + 2]), __uint_as_float(o[4 * k + 3]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->dq_free);
+    }
+    // epilogue: dV and dK rows of this tile (TMEM lane == key row)
+    if (ok && mbar_wait(&bars->done, 0, abort_flag, a.err, kTimeoutNs)) {
+      tc_fence_after();
+      const int key = u * kBK + krow;
+      const size_t orow = ((size_t)bk * p.N + key) * D + hq * (D / 2);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t ov[32], ok2[32];
+        tmem_ld32(tmem + 256 + lane_off + hq * (D / 2) + c * 32, ov);
+        tmem_ld32(tmem + 384 + lane_off + hq * (D / 2) + c * 32, ok2);
+        tmem_wait_ld();
+        if (key < p.N) {
+          uint4* dvp = reinterpret_cast<uint4*>(a.dV + orow + c * 32);
+          uint4* dkp = reinterpret_cast<uint4*>(a.dK + orow + c * 32);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            dvp[k] = make_uint4(
+                pack_bf16(__uint_as_float(ov[8 * k]), __uint_as_float(ov[8 * k + 1])),
+                pack_bf16(__uint_as_float(ov[8 * k + 2]), __uint_as_float(ov[8 * k + 3])),
+                pack_bf16(__uint_as_float(ov[8 * k + 4]), __uint_as_float(ov[8 * k + 5])),
+                pack_bf16(__uint_as_float(ov[8 * k + 6]), __uint_as_float(ov[8 * k + 7])));
+            const float s = p.scale;
+            dkp[k] = make_uint4(
+                pack_bf16(__uint_as_float(ok2[8 * k]) * s, __uint_as_float(ok2[8 * k + 1]) * s),
+                pack_bf16(__uint_as_float(ok2[8 * k + 2]) * s, __uint_as_float(ok2[8 * k + 3]) * s),
+                pack_bf16(__uint_as_float(ok2[8 * k + 4]) * s, __uint_as_float(ok2[8 * k + 5]) * s),
+                pack_bf16(__uint_as_float(ok2[8 * k + 6]) * s, __uint_as_float(ok2[8 * k + 7]) * s));
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// dQ = scale * dQacc, rounded to bf16 (8 elements per thread).
+__global__ void dq_convert_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dQ,
+                                  float scale, size_t n8) {
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
+  const float4 c = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+  reinterpret_cast<uint4*>(dQ)[i] =
+      make_uint4(pack_bf16(a.x * scale, a.y * scale), pack_bf16(a.z * scale, a.w * scale),
+                 pack_bf16(c.x * scale, c.y * scale), pack_bf16(c.z * scale, c.w * scale));
+}
+
+// D_i = dO_i . O_i, one warp per row, 16-byte loads.
+template <int D>
+__global__ void dot_rows_kernel(const __nv_bfloat16* __restrict__ O,
+                                const __nv_bfloat16* __restrict__ dO, float* __restrict__ Dvec,
+                                size_t rows) {
+  const size_t row = (size_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float s = 0.f;
+  if (lane < D / 8) {
+    const uint4 x = reinterpret_cast<const uint4*>(O + row * D)[lane];
+    const uint4 y = reinterpret_cast<const uint4*>(dO + row * D)[lane];
+    const __nv_bfloat162* xh = reinterpret_cast<const __nv_bfloat162*>(&x);
+    const __nv_bfloat162* yh = reinterpret_cast<const __nv_bfloat162*>(&y);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 xf = __bfloat1622float2(xh[k]), yf = __bfloat1622float2(yh[k]);
+      s = fmaf(xf.x, yf.x, fmaf(xf.y, yf.y, s));
+    }
+  }
+  s = warp_sum(s);
+  if (lane == 0) Dvec[row] = s;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bool make_map128(CUtensorMap* m, const void* base, int d, int rows, int heads) {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return false;
+    fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)heads};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * rows * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_bwd_typed(const BwdArgs& a, const void* Q, const void* K, const void* V,
+                             const void* O, const void* dO, void* dQ, cudaStream_t st) {
+  const Problem& p = a.p;
+  const size_t rows = (size_t)p.B * p.Hq * p.N;
+  dot_rows_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
+      (const __nv_bfloat16*)O, (const __nv_bfloat16*)dO, const_cast<float*>(a.Dvec), rows);
+  note_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_map128(&tq, Q, D, p.N, p.B * p.Hq) || !make_map128(&tk, K, D, p.N, p.B * p.Hkv) ||
+      !make_map128(&tv, V, D, p.N, p.B * p.Hkv) || !make_map128(&tdo, dO, D, p.N, p.B * p.Hq))
+    return cudaErrorInvalidValue;
+  auto kern = bwd_tc_kernel<D>;
+  const int smem = BLayout<D>::kSmemBytes;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)(p.B * p.Hkv * a.n_tiles);
+  timer_begin(GBS_OP_BWD, st);
+  kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, tdo, a);
+  timer_end(GBS_OP_BWD, st);
+  note_launch();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const size_t n8 = rows * D / 8;
+  dq_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(a.dQacc, (__nv_bfloat16*)dQ,
+                                                                    p.scale, n8);
+  note_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool bwd_tc_supported(const Problem& p) {
+  return p.dtype == GBS_BF16 && p.bs == 64 && (p.d == 64 || p.d == 128) && p.N % 64 == 0 &&
+         p.mode == GBS_TRAIN;
+}
+
+cudaError_t launch_bwd_tc(const Problem& p, const void* Q, const void* K, const void* V,
+                          const float* S, const float* slse, const void* O, const float* LSE,
+                          const void* dO, void* dQ, void* dK, void* dV, float* Dvec, float* Gblk,
+                          float* dQacc, unsigned int* err, cudaStream_t st) {
+  if (!bwd_tc_supported(p)) return cudaErrorNotSupported;
+  BwdArgs a;
+  a.p = p;
+  a.S = S;
+  a.slse = slse;
+  a.LSE = LSE;
+  a.Dvec = Dvec;
+  a.dQacc = dQacc;
+  a.Gblk = Gblk;
+  a.dK = reinterpret_cast<__nv_bfloat16*>(dK);
+  a.dV = reinterpret_cast<__nv_bfloat16*>(dV);
+  a.n_tiles = (p.Nb + 1) / 2;
+  a.err = err;
+  cudaError_t e = cudaMemsetAsync(dQacc, 0, (size_t)p.B * p.Hq * p.N * p.d * sizeof(float), st);
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(Gblk, 0, (size_t)p.B * p.Hq * p.Nb * p.Nb * sizeof(float), st);
+  if (e != cudaSuccess) return e;
+  if (p.d == 64) return launch_bwd_typed<64>(a, Q, K, V, O, dO, dQ, st);
+  return launch_bwd_typed<128>(a, Q, K, V, O, dO, dQ, st);
+}
+
+}  // namespace gbs

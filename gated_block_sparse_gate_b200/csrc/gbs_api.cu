@@ -55,7 +55,7 @@ struct FwdWs {
   size_t bytes;
 };
 struct BwdWs {
-  float *slse, *Dvec, *Gblk;
+  float *slse, *Dvec, *Gblk, *dQacc;
   size_t bytes;
 };
 struct DecWs {
@@ -88,6 +88,7 @@ BwdWs carve_bwd(const Problem& p, void* ws) {
   w.slse = c.take<float>((size_t)p.B * p.Hq * p.Nb);
   w.Dvec = c.take<float>((size_t)p.B * p.Hq * p.N);
   w.Gblk = c.take<float>((size_t)p.B * p.Hq * p.Nb * p.Nb);
+  if (bwd_tc_supported(p)) w.dQacc = c.take<float>((size_t)p.B * p.Hq * p.N * p.d);
   w.bytes = c.off;
   return w;
 }
@@ -286,6 +287,12 @@ gbs_status gbs_bwd(const gbs_params* in, const void* Q, const void* K, const voi
   cudaError_t e = launch_select(S, rows, p.Nb, p.Nb, -1, 0, false, nullptr, nullptr, nullptr,
                                 w.slse, st);
   if (e != cudaSuccess) return cuda_status(e, "gbs_bwd/select");
+  if (bwd_tc_supported(p)) {
+    e = launch_bwd_tc(p, Q, K, V, S, w.slse, O, LSE, dO, dQ, dK, dV, w.Dvec, w.Gblk, w.dQacc,
+                      err_word(ws), st);
+    if (e == cudaSuccess) e = launch_ds_finalize(p, S, w.slse, w.Gblk, dS, st);
+    return cuda_status(e, "gbs_bwd");
+  }
   return cuda_status(launch_bwd_simt(p, Q, K, V, S, w.slse, O, LSE, dO, dQ, dK, dV, dS, w.Dvec,
                                      w.Gblk, st),
                      "gbs_bwd");

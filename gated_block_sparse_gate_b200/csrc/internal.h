@@ -58,5 +58,13 @@ cudaError_t launch_fwd_tc(const Problem& p, const void* Q, const void* K, const 
                           int plan_stride, void* O, float* LSE, unsigned int* err,
                           cudaStream_t st);
 bool fwd_tc_supported(const Problem& p);
+cudaError_t launch_bwd_tc(const Problem& p, const void* Q, const void* K, const void* V,
+                          const float* S, const float* slse, const void* O, const float* LSE,
+                          const void* dO, void* dQ, void* dK, void* dV, float* Dvec, float* Gblk,
+                          float* dQacc, unsigned int* err, cudaStream_t st);
+bool bwd_tc_supported(const Problem& p);
+// dS from the tile sums G (shared by both backward paths).
+cudaError_t launch_ds_finalize(const Problem& p, const float* S, const float* slse,
+                               const float* Gblk, float* dS, cudaStream_t st);
 
 }  // namespace gbs
