@@ -193,3 +193,25 @@ def launch_count() -> int:
 def check(ws, stream=None):
     """Raises GbsError if a kernel recorded a device-side error in ``ws``."""
     _check(load_library().gbs_check(_ptr(ws), _stream(stream)), "gbs_check")
+
+
+def decode_noalloc(q, Kc, Vc, S, L=None, block=64, topk=32, scale=0.0, num_splits=0, out=None,
+                   lse=None, stream=None):
+    """gbs_decode_noalloc: the decode with the library's own static scratch.
+
+    For callers that cannot allocate device memory while decoding; see
+    include/gbs.h for the limits and the sharing rules.
+    """
+    lib = load_library()
+    f = lib.gbs_decode_noalloc
+    vp = ctypes.c_void_p
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.POINTER(Params), vp, vp, vp, vp, vp, vp, ctypes.c_int, vp]
+    B, Hq, d = q.shape
+    L = Kc.shape[2] if L is None else L
+    p = make_params(B, Hq, Kc.shape[1], L, d, block, topk, "sparse", q.dtype, scale)
+    O = out if out is not None else torch.empty_like(q)
+    LSE = lse if lse is not None else torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    _check(f(ctypes.byref(p), _ptr(q), _ptr(Kc), _ptr(Vc), _ptr(S), _ptr(O), _ptr(LSE), num_splits,
+             _stream(stream)), "gbs_decode_noalloc")
+    return O, LSE

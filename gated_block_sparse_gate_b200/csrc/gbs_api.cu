@@ -161,6 +161,7 @@ unsigned int* err_word(void* ws) { return reinterpret_cast<unsigned int*>(ws); }
 }  // namespace
 
 namespace gbs {
+void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
 void note_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 void timer_begin(int op, cudaStream_t st) {
   if (g_timer[op][0]) cudaEventRecord(g_timer[op][0], st);

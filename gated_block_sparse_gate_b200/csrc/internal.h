@@ -12,6 +12,8 @@ namespace gbs {
 // Bookkeeping shared by all launchers: every kernel launch is counted, and
 // the main kernel of an op is bracketed by the caller's timer events if set.
 void note_launch(int n = 1);
+// Sets the text returned by gbs_last_error() on the calling thread.
+void set_last_error(const char* msg);
 void timer_begin(int op, cudaStream_t st);
 void timer_end(int op, cudaStream_t st);
 

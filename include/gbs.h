@@ -168,6 +168,28 @@ GBS_API gbs_status gbs_set_timer(int op, void* start, void* stop);
 /* Total number of CUDA kernels this library has launched in this process. */
 GBS_API uint64_t gbs_launch_count(void);
 
+/* Bytes of device scratch that gbs_decode_noalloc keeps in the library. */
+#define GBS_DECODE_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* Sparse decode without a workspace (no counterpart in the paper: this is a
+ * convenience of this library, not part of the method).
+ * Same inputs, outputs and results as gbs_decode, for callers that cannot
+ * allocate device memory when they decode, e.g. a serving loop whose device
+ * memory is reserved up front by another allocator, or one that must not call
+ * cudaMalloc on its hot path because that call can synchronise the device.
+ * The Top-K lists and per-split partials live in a static device array of
+ * GBS_DECODE_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds
+ * until the process exits. The first call on each device looks up that
+ * array's address (cudaGetSymbolAddress, with the device current); make that
+ * first call before any stream capture. Calls on one device share the array:
+ * calls that overlap on the GPU race and must be serialised by the caller.
+ * Rejects, with GBS_ERR_INVALID_ARG and a gbs_last_error() message, any size
+ * whose scratch (about B*Hq*(8*topk + 8 + splits*(4*d + 8)) bytes, splits <= 8)
+ * exceeds the array; allocates and frees nothing. */
+GBS_API gbs_status gbs_decode_noalloc(const gbs_params* p, const void* q, const void* Kc,
+                                      const void* Vc, const float* S, void* O, float* LSE,
+                                      int num_splits, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
