@@ -260,6 +260,10 @@ gbs_status gbs_fwd(const gbs_params* in, const void* Q, const void* K, const voi
   cudaError_t e = launch_select(S, rows, p.Nb, p.Nb, -1, p.topk, sparse, w.sel.idx, w.sel.cnt,
                                 w.sel.logg, sparse ? nullptr : w.sel.slse, st);
   if (e != cudaSuccess) return cuda_status(e, "gbs_fwd/select");
+  if (fwd_tc2_supported(p)) {
+    e = launch_fwd_tc2(p, Q, K, V, S, w.sel.slse, O, LSE, err_word(ws), st);
+    if (e != cudaErrorNotSupported) return cuda_status(e, "gbs_fwd/attention");
+  }
   if (p.dtype == GBS_BF16 && fwd_tc_supported(p)) {
     e = launch_fwd_tc(p, Q, K, V, S, w.sel, w.plan, (int)plan_stride(p), O, LSE, err_word(ws), st);
     if (e != cudaErrorNotSupported) return cuda_status(e, "gbs_fwd/attention");

@@ -60,6 +60,11 @@ cudaError_t launch_fwd_tc(const Problem& p, const void* Q, const void* K, const 
                           int plan_stride, void* O, float* LSE, unsigned int* err,
                           cudaStream_t st);
 bool fwd_tc_supported(const Problem& p);
+// Training mode with an even q-heads-per-kv-head ratio: two query tiles per CTA.
+cudaError_t launch_fwd_tc2(const Problem& p, const void* Q, const void* K, const void* V,
+                           const float* S, const float* slse, void* O, float* LSE,
+                           unsigned int* err, cudaStream_t st);
+bool fwd_tc2_supported(const Problem& p);
 cudaError_t launch_bwd_tc(const Problem& p, const void* Q, const void* K, const void* V,
                           const float* S, const float* slse, const void* O, const float* LSE,
                           const void* dO, void* dQ, void* dK, void* dV, float* Dvec, float* Gblk,
