@@ -20,8 +20,10 @@
 //                  per-warp sums of dZ added into G
 //   dV += P^T dO, dK += dZ^T Q      (A from TMEM, B = dO / Q MN-major)
 //   dQ  = dZ K                      (A = dZ^T smem MN-major, B = K MN-major;
-//                                    TMEM, drained by vector reductions into
-//                                    an fp32 accumulator in the workspace)
+//                                    TMEM; each warp stages its 32 x D/2 part
+//                                    in the step's now-consumed Q / dO smem
+//                                    stage and a TMA tensor reduce-add adds it
+//                                    into the fp32 accumulator at L2)
 // TMEM (512 columns): R0 = S^T / P^T / dQ, R1 = dP^T / dZ^T, dV, dK. The bf16
 // P^T and dZ^T of query half h are stored over the first 32 columns of that
 // half's own 64 S^T / dP^T columns.
@@ -57,7 +59,7 @@ struct BLayout {
   static constexpr int kQOff = kVOff + kTile;
   static constexpr int kdOOff = kQOff + kQStages * kTile;
   static constexpr int kZOff = kdOOff + kQStages * kTile;   // dZ^T: 128 keys x 128 queries
-  static constexpr int kVecOff = kZOff + 2 * kChunk;        // (lse2, D) per query, per stage
+  static constexpr int kVecOff = kZOff + 2 * kChunk;        // LSE[128], D[128] per stage
   static constexpr int kBarOff = kVecOff + kQStages * kBQ * 8;
   static constexpr int kSmemBytes = kBarOff + 256;
 };
@@ -65,7 +67,7 @@ struct BLayout {
 struct BBarriers {
   uint64_t kv_full;
   uint64_t q_full[kQStages];
-  uint64_t q_empty[kQStages];
+  uint64_t st_drained[kQStages];  // the stage's dQ staging has been read by the TMA
   uint64_t st_full;
   uint64_t p_full;
   uint64_t dq_full;
@@ -106,7 +108,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-              BwdArgs a) {
+              const __grid_constant__ CUtensorMap tmdQ, BwdArgs a) {
   using L = BLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {  // the swizzled tiles need 1024-byte alignment
@@ -128,7 +130,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     mbar_init(&bars->kv_full, 1);
     for (int s = 0; s < kQStages; ++s) {
       mbar_init(&bars->q_full[s], 1);
-      mbar_init(&bars->q_empty[s], 1);
+      mbar_init(&bars->st_drained[s], kComputeWarps);
     }
     mbar_init(&bars->st_full, 1);
     mbar_init(&bars->p_full, kComputeWarps * 32);
@@ -147,7 +149,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort_flag = &bars->abort_flag;
-  float2* vecs = reinterpret_cast<float2*>(smem + L::kVecOff);
+  float* vecs = reinterpret_cast<float*>(smem + L::kVecOff);
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
@@ -156,49 +158,44 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       prefetch_tmap(&tmdO);
+      prefetch_tmap(&tmdQ);
       mbar_arrive_expect_tx(&bars->kv_full, 2 * L::kTile);
       for (int ch = 0; ch < L::kChunks; ++ch) {
         tma_load_3d(smem + L::kKOff + ch * kChunk, &tmK, &bars->kv_full, ch * 64, u * kBK, bk);
         tma_load_3d(smem + L::kVOff + ch * kChunk, &tmV, &bars->kv_full, ch * 64, u * kBK, bk);
       }
     }
-    int issued = 0;
-    for (int j = 0; j < n_steps; ++j) {
-      const int st = j % kQStages;
-      int ok = 1;
-      if (lane == 0 && j >= kQStages)
-        ok = mbar_wait(&bars->q_empty[st], ((j / kQStages) - 1) & 1, abort_flag, a.err, kTimeoutNs);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      const int hh = j / per_head, t = u + j % per_head;
-      const int bh = b * p.Hq + kvh * p.G + hh;
-      const int q0 = t * kBQ;
-      float2* vec = vecs + st * kBQ;
-      for (int i = lane; i < kBQ; i += 32) {
-        const int q = q0 + i;
-        float2 v = make_float2(INFINITY, 0.f);  // rows past the end contribute nothing
-        if (q < p.N) {
-          const size_t idx = (size_t)bh * p.N + q;
-          v = make_float2(__ldg(a.LSE + idx) * GBS_LOG2E, __ldg(a.Dvec + idx));
-        }
-        vec[i] = v;
-      }
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&bars->q_full[st], 2 * L::kTile);
+    if (lane == 0) {
+      int issued = 0;
+      for (int j = 0; j < n_steps; ++j) {
+        const int st = j % kQStages;
+        // the stage is free once step j-2's MMAs are done and its dQ staging was read
+        if (j >= kQStages &&
+            !mbar_wait(&bars->st_drained[st], ((j / kQStages) - 1) & 1, abort_flag, a.err, kTimeoutNs))
+          break;
+        const int hh = j / per_head, t = u + j % per_head;
+        const int bh = b * p.Hq + kvh * p.G + hh;
+        const int q0 = t * kBQ;
+        // rows past the end are never read: a half tile past N is fully masked
+        const int nvalid = (p.N - q0) < kBQ ? (p.N - q0) : kBQ;
+        float* lse_s = vecs + st * 2 * kBQ;
+        mbar_arrive_expect_tx(&bars->q_full[st], 2 * L::kTile + 2 * nvalid * 4);
         uint8_t* qs = smem + L::kQOff + st * L::kTile;
         uint8_t* ds = smem + L::kdOOff + st * L::kTile;
         for (int ch = 0; ch < L::kChunks; ++ch) {
           tma_load_3d(qs + ch * kChunk, &tmQ, &bars->q_full[st], ch * 64, q0, bh);
           tma_load_3d(ds + ch * kChunk, &tmdO, &bars->q_full[st], ch * 64, q0, bh);
         }
+        bulk_load(lse_s, a.LSE + (size_t)bh * p.N + q0, nvalid * 4, &bars->q_full[st]);
+        bulk_load(lse_s + kBQ, a.Dvec + (size_t)bh * p.N + q0, nvalid * 4, &bars->q_full[st]);
+        issued = j + 1;
       }
-      issued = j + 1;
-    }
-    if (lane == 0 && *abort_flag) {
-      // let loads still in flight land before the CTA exits
-      mbar_wait(&bars->kv_full, 0, abort_flag, nullptr, 1000000ull);
-      for (int j = issued - kQStages < 0 ? 0 : issued - kQStages; j < issued; ++j)
-        mbar_wait(&bars->q_full[j % kQStages], (j / kQStages) & 1, abort_flag, nullptr, 1000000ull);
+      if (*abort_flag) {
+        // let loads still in flight land before the CTA exits
+        mbar_wait(&bars->kv_full, 0, abort_flag, nullptr, 1000000ull);
+        for (int j = issued - kQStages < 0 ? 0 : issued - kQStages; j < issued; ++j)
+          mbar_wait(&bars->q_full[j % kQStages], (j / kQStages) & 1, abort_flag, nullptr, 1000000ull);
+      }
     }
   } else if (warp == 9) {
     // -------------------------------------------------------------- MMA issuer
@@ -255,7 +252,6 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           mma_ss(R0, sdesc_sw128(z_addr + ks * 2048, kChunk, 1024),
                  sdesc_sw128(k_addr + ks * 2048, kChunk, 1024), idQ, ks > 0 ? 1u : 0u);
         mma_commit(&bars->dq_full);
-        mma_commit(&bars->q_empty[st]);
         if (j + 1 < n_steps && !issue_dp(j + 1)) break;
       }
       mma_commit(&bars->done);
@@ -291,8 +287,11 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         break;
       }
       tc_fence_after();
-      const float2* vec = vecs + st * kBQ + hq * 64;
-      float g = 0.f;
+      const float* lse_s = vecs + st * 2 * kBQ + hq * 64;  // natural-log LSE
+      const float* dvec_s = lse_s + kBQ;                   // D = dO . O
+      const f32x2 scv = f2_make(sc, sc), biasv = f2_make(bias2, bias2);
+      const f32x2 nlog2e = f2_make(-GBS_LOG2E, -GBS_LOG2E);
+      f32x2 g2 = f2_make(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {  // two chunks of 32 query columns
         const uint32_t col = hq * 64 + c * 32;
@@ -305,20 +304,31 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           for (int k = 0; k < 16; ++k) pp[k] = zz[k] = 0u;
         } else {
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            float pr[2], dz[2];
+          for (int k = 0; k < 32; k += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(lse_s + c * 32 + k);
+            const float4 d4 = *reinterpret_cast<const float4*>(dvec_s + c * 32 + k);
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int i = 2 * k + e;
-              const float2 ld = vec[c * 32 + i];
-              float x = fmaf(__uint_as_float(sv[i]), sc, bias2 - ld.x);
-              if (mode == kCausal && c * 32 + i < jloc) x = -INFINITY;
-              pr[e] = ex2(x);
-              dz[e] = pr[e] * (__uint_as_float(dv[i]) - ld.y);
+            for (int e = 0; e < 4; e += 2) {
+              const int i = k + e;
+              // x = scale*log2e*s + bias*log2e - LSE*log2e, two columns at a time
+              f32x2 x2 = f2_fma(f2_make(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), scv, biasv);
+              x2 = f2_fma(e == 0 ? f2_make(l4.x, l4.y) : f2_make(l4.z, l4.w), nlog2e, x2);
+              float x0, x1;
+              f2_split(x2, x0, x1);
+              if (mode == kCausal) {
+                if (c * 32 + i < jloc) x0 = -INFINITY;
+                if (c * 32 + i + 1 < jloc) x1 = -INFINITY;
+              }
+              const float p0 = ex2(x0), p1 = ex2(x1);
+              const f32x2 dd = f2_sub(f2_make(__uint_as_float(dv[i]), __uint_as_float(dv[i + 1])),
+                                      e == 0 ? f2_make(d4.x, d4.y) : f2_make(d4.z, d4.w));
+              const f32x2 dz = f2_mul(f2_make(p0, p1), dd);
+              g2 = f2_add(g2, dz);
+              float dz0, dz1;
+              f2_split(dz, dz0, dz1);
+              pp[i / 2] = pack_bf16(p0, p1);
+              zz[i / 2] = pack_bf16(dz0, dz1);
             }
-            g += dz[0] + dz[1];
-            pp[k] = pack_bf16(pr[0], pr[1]);
-            zz[k] = pack_bf16(dz[0], dz[1]);
           }
         }
         // packed outputs stay inside this warp's own 64 columns of S^T / dP^T
@@ -333,6 +343,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
               make_uint4(zz[4 * gi], zz[4 * gi + 1], zz[4 * gi + 2], zz[4 * gi + 3]);
         }
       }
+      float g, g_hi;
+      f2_split(g2, g, g_hi);
+      g += g_hi;
       g = warp_sum(g);
       if (lane == 0 && mode != kMasked) atomicAdd(a.Gblk + ((size_t)bh * p.Nb + r) * p.Nb + cj, g);
       tmem_wait_st();
@@ -346,23 +359,38 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         break;
       }
       tc_fence_after();
-      const int qrow = t * kBQ + krow;
-      float* dst = a.dQacc + ((size_t)bh * p.N + qrow) * D + hq * (D / 2);
+      // stage this warp's 32 rows x D/2 columns of dQ (128-byte swizzled boxes
+      // of 32 x 32 fp32) in the step's Q (hq 0) or dO (hq 1) stage, which every
+      // MMA of the step has finished reading
+      const int qrow0 = t * kBQ + quad * 32;
+      uint8_t* stg = smem + (hq == 0 ? L::kQOff : L::kdOOff) + st * L::kTile + quad * (D / 2) * 128;
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
+      for (int bx = 0; bx < D / 64; ++bx) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_off + hq * (D / 2) + c * 32, o);
+        tmem_ld32(tmem + lane_off + hq * (D / 2) + bx * 32, o);
         tmem_wait_ld();
-        if (qrow < p.N) {
+        uint8_t* row = stg + bx * 4096 + lane * 128;
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            red_add_v4(dst + c * 32 + 4 * k, __uint_as_float(o[4 * k]), __uint_as_float(o[4 * k + 1]),
-                       __uint_as_float(o[4 * k + 2]), __uint_as_float(o[4 * k + 3]));
-        }
+        for (int gi = 0; gi < 8; ++gi)
+          *reinterpret_cast<uint4*>(row + ((gi ^ (lane & 7)) << 4)) =
+              make_uint4(o[4 * gi], o[4 * gi + 1], o[4 * gi + 2], o[4 * gi + 3]);
       }
+      fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars->dq_free);
+      mbar_arrive(&bars->dq_free);  // TMEM is free; the reduction proceeds from smem
+      __syncwarp();
+      if (lane == 0) {
+        if (qrow0 < p.N) {
+#pragma unroll
+          for (int bx = 0; bx < D / 64; ++bx)
+            tma_reduce_add_2d(&tmdQ, hq * (D / 2) + bx * 32, bh * p.N + qrow0, stg + bx * 4096);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+        }
+        mbar_arrive(&bars->st_drained[st]);
+      }
     }
+    if (lane == 0) bulk_wait_group0();  // reductions reach global memory before exit
     // epilogue: dV and dK rows of this tile (TMEM lane == key row)
     if (ok && mbar_wait(&bars->done, 0, abort_flag, a.err, kTimeoutNs)) {
       tc_fence_after();
@@ -464,6 +492,27 @@ bool make_map128(CUtensorMap* m, const void* base, int d, int rows, int heads) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// dQ accumulator, fp32 rows of D: dims (D, rows), 32 x 32 boxes, 128-byte swizzle.
+bool make_map_dq(CUtensorMap* m, const void* base, int d, size_t rows) {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return false;
+    fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)d * 4};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D>
 cudaError_t launch_bwd_typed(const BwdArgs& a, const void* Q, const void* K, const void* V,
                              const void* O, const void* dO, void* dQ, cudaStream_t st) {
@@ -474,9 +523,10 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, const void* Q, const void* K, con
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   if (!make_map128(&tq, Q, D, p.N, p.B * p.Hq) || !make_map128(&tk, K, D, p.N, p.B * p.Hkv) ||
-      !make_map128(&tv, V, D, p.N, p.B * p.Hkv) || !make_map128(&tdo, dO, D, p.N, p.B * p.Hq))
+      !make_map128(&tv, V, D, p.N, p.B * p.Hkv) || !make_map128(&tdo, dO, D, p.N, p.B * p.Hq) ||
+      !make_map_dq(&tdq, a.dQacc, D, rows))
     return cudaErrorInvalidValue;
   auto kern = bwd_tc_kernel<D>;
   const int smem = BLayout<D>::kSmemBytes;
@@ -484,7 +534,7 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, const void* Q, const void* K, con
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)(p.B * p.Hkv * a.n_tiles);
   timer_begin(GBS_OP_BWD, st);
-  kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, tdo, a);
+  kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, tdo, tdq, a);
   timer_end(GBS_OP_BWD, st);
   note_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
