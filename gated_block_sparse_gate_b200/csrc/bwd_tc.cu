@@ -22,8 +22,8 @@
 //   dQ  = dZ K                      (A = dZ^T smem MN-major, B = K MN-major;
 //                                    TMEM; each warp stages its 32 x D/2 part
 //                                    in the step's now-consumed Q / dO smem
-//                                    stage and a TMA tensor reduce-add adds it
-//                                    into the fp32 accumulator at L2)
+//                                    stage and the TMA warp issues tensor
+//                                    reduce-adds into the fp32 accumulator)
 // TMEM (512 columns): R0 = S^T / P^T / dQ, R1 = dP^T / dZ^T, dV, dK. The bf16
 // P^T and dZ^T of query half h are stored over the first 32 columns of that
 // half's own 64 S^T / dP^T columns.
@@ -67,7 +67,7 @@ struct BLayout {
 struct BBarriers {
   uint64_t kv_full;
   uint64_t q_full[kQStages];
-  uint64_t st_drained[kQStages];  // the stage's dQ staging has been read by the TMA
+  uint64_t staged[kQStages];  // every compute warp has staged the step's dQ in this stage
   uint64_t st_full;
   uint64_t p_full;
   uint64_t dq_full;
@@ -130,7 +130,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     mbar_init(&bars->kv_full, 1);
     for (int s = 0; s < kQStages; ++s) {
       mbar_init(&bars->q_full[s], 1);
-      mbar_init(&bars->st_drained[s], kComputeWarps);
+      mbar_init(&bars->staged[s], kComputeWarps);
     }
     mbar_init(&bars->st_full, 1);
     mbar_init(&bars->p_full, kComputeWarps * 32);
@@ -166,13 +166,38 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       }
     }
     if (lane == 0) {
+      // adds step jj's staged dQ (8 warps x 32 rows x D/2 columns) into the accumulator
+      auto reduce_step = [&](int jj) -> bool {
+        const int sj = jj % kQStages;
+        if (!mbar_wait(&bars->staged[sj], (jj / kQStages) & 1, abort_flag, a.err, kTimeoutNs))
+          return false;
+        const int t = u + jj % per_head;
+        const int bh = b * p.Hq + kvh * p.G + jj / per_head;
+#pragma unroll 1
+        for (int w = 0; w < kComputeWarps; ++w) {
+          const int quad = w & 3, hq = w >> 2;
+          const int qrow0 = t * kBQ + quad * 32;
+          if (qrow0 >= p.N) continue;
+          const uint8_t* stg =
+              smem + (hq == 0 ? L::kQOff : L::kdOOff) + sj * L::kTile + quad * (D / 2) * 128;
+          for (int bx = 0; bx < D / 64; ++bx)
+            tma_reduce_add_2d(&tmdQ, hq * (D / 2) + bx * 32, bh * p.N + qrow0, stg + bx * 4096);
+        }
+        bulk_commit_group();
+        return true;
+      };
       int issued = 0;
+      bool ok = true;
       for (int j = 0; j < n_steps; ++j) {
         const int st = j % kQStages;
-        // the stage is free once step j-2's MMAs are done and its dQ staging was read
-        if (j >= kQStages &&
-            !mbar_wait(&bars->st_drained[st], ((j / kQStages) - 1) & 1, abort_flag, a.err, kTimeoutNs))
-          break;
+        // the stage is free once step j-2's MMAs are done and its staged dQ was read
+        if (j >= kQStages) {
+          if (!reduce_step(j - kQStages)) {
+            ok = false;
+            break;
+          }
+          bulk_wait_group_read0();
+        }
         const int hh = j / per_head, t = u + j % per_head;
         const int bh = b * p.Hq + kvh * p.G + hh;
         const int q0 = t * kBQ;
@@ -190,6 +215,10 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         bulk_load(lse_s + kBQ, a.Dvec + (size_t)bh * p.N + q0, nvalid * 4, &bars->q_full[st]);
         issued = j + 1;
       }
+      if (ok)
+        for (int jj = n_steps - kQStages < 0 ? 0 : n_steps - kQStages; jj < n_steps; ++jj)
+          if (!reduce_step(jj)) break;
+      bulk_wait_group0();  // reductions reach global memory before the CTA exits
       if (*abort_flag) {
         // let loads still in flight land before the CTA exits
         mbar_wait(&bars->kv_full, 0, abort_flag, nullptr, 1000000ull);
@@ -362,7 +391,6 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       // stage this warp's 32 rows x D/2 columns of dQ (128-byte swizzled boxes
       // of 32 x 32 fp32) in the step's Q (hq 0) or dO (hq 1) stage, which every
       // MMA of the step has finished reading
-      const int qrow0 = t * kBQ + quad * 32;
       uint8_t* stg = smem + (hq == 0 ? L::kQOff : L::kdOOff) + st * L::kTile + quad * (D / 2) * 128;
 #pragma unroll
       for (int bx = 0; bx < D / 64; ++bx) {
@@ -379,18 +407,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tc_fence_before();
       mbar_arrive(&bars->dq_free);  // TMEM is free; the reduction proceeds from smem
       __syncwarp();
-      if (lane == 0) {
-        if (qrow0 < p.N) {
-#pragma unroll
-          for (int bx = 0; bx < D / 64; ++bx)
-            tma_reduce_add_2d(&tmdQ, hq * (D / 2) + bx * 32, bh * p.N + qrow0, stg + bx * 4096);
-          bulk_commit_group();
-          bulk_wait_group_read0();
-        }
-        mbar_arrive(&bars->st_drained[st]);
-      }
+      if (lane == 0) mbar_arrive(&bars->staged[st]);  // the producer issues the reduction
     }
-    if (lane == 0) bulk_wait_group0();  // reductions reach global memory before exit
     // epilogue: dV and dK rows of this tile (TMEM lane == key row)
     if (ok && mbar_wait(&bars->done, 0, abort_flag, a.err, kTimeoutNs)) {
       tc_fence_after();
