@@ -240,6 +240,57 @@ def bench_training(w, steps, warmup, rank, dev, peaks):
     return res
 
 
+def bench_training_long(dev, peaks, reps=5):
+    """Long-context training step (N=32768, 512 blocks): forward + backward."""
+    from gated_block_sparse_gate_b200 import binding as gb
+
+    w = WORKLOADS["train_bf16_n32768"]
+    x = make_prefill_inputs(w)
+    d = {k: v.to(dev) for k, v in x.items()}
+    del x
+    Q, K, V, S, dO = d["Q"], d["K"], d["V"], d["S"], d["dO"]
+    pf = gb.make_params(w.B, w.Hq, w.Hkv, w.N, w.d, w.block, 0, "train", Q.dtype)
+    ws_f = gb.alloc_workspace(pf, gb.OP_FWD, dev)
+    ws_b = gb.alloc_workspace(pf, gb.OP_BWD, dev)
+    O = torch.empty_like(Q)
+    LSE = torch.empty(Q.shape[:3], dtype=torch.float32, device=dev)
+    grads = (torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V), torch.empty_like(S))
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        gb.forward(Q, K, V, S, mode="train", out=O, lse=LSE, ws=ws_f)
+        gb.backward(Q, K, V, S, O, LSE, dO, grads=grads, ws=ws_b)
+
+    for _ in range(2):
+        step()
+    a0, a1 = _events(reps), _events(reps)
+    f0, f1, b0, b1 = _events(reps), _events(reps), _events(reps), _events(reps)
+    torch.cuda.synchronize()
+    for i in range(reps):
+        flush.zero_()
+        gb.set_timer(gb.OP_FWD, f0[i], f1[i])
+        gb.set_timer(gb.OP_BWD, b0[i], b1[i])
+        a0[i].record()
+        step()
+        a1[i].record()
+    torch.cuda.synchronize()
+    gb.set_timer(gb.OP_FWD)
+    gb.set_timer(gb.OP_BWD)
+    gb.check(ws_f)
+    gb.check(ws_b)
+    ms = statistics.mean(a.elapsed_time(b) for a, b in zip(a0, a1))
+    fms = statistics.mean(a.elapsed_time(b) for a, b in zip(f0, f1))
+    bms = statistics.mean(a.elapsed_time(b) for a, b in zip(b0, b1))
+    P = train_pairs_per_head(w.Nb, w.block) * w.B * w.Hq
+    fl_f, fl_fb = 4.0 * w.d * P, 14.0 * w.d * P
+    del d, grads, O
+    torch.cuda.empty_cache()
+    return {"ms_per_step": ms, "tflops": fl_fb / ms / 1e9,
+            "pct_of_bf16_peak": 100.0 * fl_fb / ms / 1e9 / peaks["bf16_tflops"],
+            "fwd_kernel_ms": fms, "fwd_kernel_tflops": fl_f / fms / 1e9,
+            "bwd_main_ms": bms, "bwd_main_tflops": (fl_fb - fl_f) / bms / 1e9}
+
+
 def bench_sparse_prefill(dev, peaks, reps=5):
     """Sparse prefill N=65536, Top-K sweep; forward only."""
     from gated_block_sparse_gate_b200 import binding as gb
@@ -429,6 +480,7 @@ def main(argv=None):
     e2e_ms = gdist.max_over_ranks(r["e2e"]["ms"], dev)
     extra = {}
     if ws == 1 and not args.no_extra:
+        extra["train_bf16_n32768"] = bench_training_long(dev, peaks)
         extra["sparse_prefill_bf16_n65536"] = bench_sparse_prefill(dev, peaks)
         extra["sparse_decode_bf16_b64_l131072"] = bench_decode(dev, peaks)
     if rank == 0:

@@ -24,9 +24,13 @@
 //                                    in the step's now-consumed Q / dO smem
 //                                    stage and the TMA warp issues tensor
 //                                    reduce-adds into the fp32 accumulator)
-// TMEM (512 columns): R0 = S^T / P^T / dQ, R1 = dP^T / dZ^T, dV, dK. The bf16
+// TMEM (512 columns): R0 = S^T / P^T, R1 = dP^T / dZ^T / dQ, dV, dK. The bf16
 // P^T and dZ^T of query half h are stored over the first 32 columns of that
 // half's own 64 S^T / dP^T columns.
+// The compute warps work in two phases per step: phase A turns S^T into P^T
+// (the dV MMA starts on it), phase B turns dP^T into dZ^T (dK and dQ start).
+// The next step's S^T is issued as soon as dQ is issued, so its phase A
+// overlaps the drain of dQ and the dP^T MMA.
 // Warps: 0-7 compute (lane quadrant w%4, query/column half w/4), 8 TMA,
 // 9 TMEM allocator + MMA issuer. Every mbarrier wait is bounded.
 #include <cuda.h>
@@ -68,8 +72,10 @@ struct BBarriers {
   uint64_t kv_full;
   uint64_t q_full[kQStages];
   uint64_t staged[kQStages];  // every compute warp has staged the step's dQ in this stage
-  uint64_t st_full;
-  uint64_t p_full;
+  uint64_t s_full;   // S^T of the step landed in R0
+  uint64_t dp_full;  // dP^T of the step landed in R1
+  uint64_t pa_full;  // P^T written (dV can start)
+  uint64_t pb_full;  // dZ^T written to TMEM and smem (dK, dQ can start)
   uint64_t dq_full;
   uint64_t dq_free;
   uint64_t done;
@@ -132,8 +138,10 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       mbar_init(&bars->q_full[s], 1);
       mbar_init(&bars->staged[s], kComputeWarps);
     }
-    mbar_init(&bars->st_full, 1);
-    mbar_init(&bars->p_full, kComputeWarps * 32);
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->dp_full, 1);
+    mbar_init(&bars->pa_full, kComputeWarps * 32);
+    mbar_init(&bars->pb_full, kComputeWarps * 32);
     mbar_init(&bars->dq_full, 1);
     mbar_init(&bars->dq_free, kComputeWarps * 32);
     mbar_init(&bars->done, 1);
@@ -236,11 +244,25 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       const uint32_t k_addr = smem_u32(smem + L::kKOff), v_addr = smem_u32(smem + L::kVOff);
       const uint32_t z_addr = smem_u32(smem + L::kZOff);
       bool ok = mbar_wait(&bars->kv_full, 0, abort_flag, a.err, kTimeoutNs);
-      auto issue_dp = [&](int j) -> bool {
+      // S^T_j = K Q_j^T -> R0 (waits for the step's Q / dO / LSE / D)
+      auto issue_s = [&](int j) -> bool {
         const int st = j % kQStages;
         if (!mbar_wait(&bars->q_full[st], (j / kQStages) & 1, abort_flag, a.err, kTimeoutNs))
           return false;
         tc_fence_after();
+        const uint32_t q_addr = smem_u32(smem + L::kQOff + st * L::kTile);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const int ch = ks >> 2, kk = ks & 3;
+          mma_ss(R0, sdesc_sw128(k_addr + ch * kChunk + kk * 32, 16, 1024),
+                 sdesc_sw128(q_addr + ch * kChunk + kk * 32, 16, 1024), idST, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars->s_full);
+        return true;
+      };
+      // dP^T_j = V dO_j^T -> R1
+      auto issue_dp = [&](int j) {
+        const int st = j % kQStages;
         const uint32_t do_addr = smem_u32(smem + L::kdOOff + st * L::kTile);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
@@ -248,40 +270,43 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           mma_ss(R1, sdesc_sw128(v_addr + ch * kChunk + kk * 32, 16, 1024),
                  sdesc_sw128(do_addr + ch * kChunk + kk * 32, 16, 1024), idST, ks > 0 ? 1u : 0u);
         }
-        return true;
+        mma_commit(&bars->dp_full);
       };
-      if (ok) ok = issue_dp(0);
+      if (ok) ok = issue_s(0);
+      if (ok) issue_dp(0);
       for (int j = 0; ok && j < n_steps; ++j) {
         const int st = j % kQStages;
         const uint32_t q_addr = smem_u32(smem + L::kQOff + st * L::kTile);
         const uint32_t do_addr = smem_u32(smem + L::kdOOff + st * L::kTile);
-        if (j > 0) {
-          if (!mbar_wait(&bars->dq_free, (j - 1) & 1, abort_flag, a.err, kTimeoutNs)) break;
-          tc_fence_after();
-        }
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const int ch = ks >> 2, kk = ks & 3;
-          mma_ss(R0, sdesc_sw128(k_addr + ch * kChunk + kk * 32, 16, 1024),
-                 sdesc_sw128(q_addr + ch * kChunk + kk * 32, 16, 1024), idST, ks > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars->st_full);
-        if (!mbar_wait(&bars->p_full, j & 1, abort_flag, a.err, kTimeoutNs)) break;
-        tc_fence_after();
         // P^T / dZ^T of query half hq sit in columns [64 hq, 64 hq + 32) of R0 / R1
+        if (!mbar_wait(&bars->pa_full, j & 1, abort_flag, a.err, kTimeoutNs)) break;
+        tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < kBQ / 16; ++ks) {
-          const uint32_t acc = (j > 0 || ks > 0) ? 1u : 0u;
           const uint32_t acol = (ks >> 2) * 64 + (ks & 3) * 8;
-          mma_ts(TdV, R0 + acol, sdesc_sw128(do_addr + ks * 2048, kChunk, 1024), idKV, acc);
-          mma_ts(TdK, R1 + acol, sdesc_sw128(q_addr + ks * 2048, kChunk, 1024), idKV, acc);
+          mma_ts(TdV, R0 + acol, sdesc_sw128(do_addr + ks * 2048, kChunk, 1024), idKV,
+                 (j > 0 || ks > 0) ? 1u : 0u);
         }
+        if (!mbar_wait(&bars->pb_full, j & 1, abort_flag, a.err, kTimeoutNs)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < kBQ / 16; ++ks) {
+          const uint32_t acol = (ks >> 2) * 64 + (ks & 3) * 8;
+          mma_ts(TdK, R1 + acol, sdesc_sw128(q_addr + ks * 2048, kChunk, 1024), idKV,
+                 (j > 0 || ks > 0) ? 1u : 0u);
+        }
+        // dQ_j = dZ_j K -> R1 (after dK_j has read dZ^T from R1: MMAs run in order)
 #pragma unroll
         for (int ks = 0; ks < kBK / 16; ++ks)
-          mma_ss(R0, sdesc_sw128(z_addr + ks * 2048, kChunk, 1024),
+          mma_ss(R1, sdesc_sw128(z_addr + ks * 2048, kChunk, 1024),
                  sdesc_sw128(k_addr + ks * 2048, kChunk, 1024), idQ, ks > 0 ? 1u : 0u);
         mma_commit(&bars->dq_full);
-        if (j + 1 < n_steps && !issue_dp(j + 1)) break;
+        if (j + 1 < n_steps) {
+          if (!issue_s(j + 1)) break;  // R0 is free once dV_j has read P^T_j
+          if (!mbar_wait(&bars->dq_free, j & 1, abort_flag, a.err, kTimeoutNs)) break;
+          tc_fence_after();
+          issue_dp(j + 1);  // R1 is free once dQ_j has been drained
+        }
       }
       mma_commit(&bars->done);
       mbar_wait(&bars->done, 0, abort_flag, a.err, kTimeoutNs);
@@ -310,7 +335,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const size_t row = (size_t)bh * p.Nb + r;
         bias2 = (__ldg(a.S + row * p.Nb + cj) - __ldg(a.slse + row)) * GBS_LOG2E;
       }
-      if (!mbar_wait(&bars->st_full, j & 1, abort_flag, a.err, kTimeoutNs) ||
+      if (!mbar_wait(&bars->s_full, j & 1, abort_flag, a.err, kTimeoutNs) ||
           !mbar_wait(&bars->q_full[st], (j / kQStages) & 1, abort_flag, a.err, kTimeoutNs)) {
         ok = false;
         break;
@@ -320,26 +345,23 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       const float* dvec_s = lse_s + kBQ;                   // D = dO . O
       const f32x2 scv = f2_make(sc, sc), biasv = f2_make(bias2, bias2);
       const f32x2 nlog2e = f2_make(-GBS_LOG2E, -GBS_LOG2E);
-      f32x2 g2 = f2_make(0.f, 0.f);
+      // phase A: P^T = exp2(scale log2e s + bias - LSE log2e) from S^T alone
+      float pr[64];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {  // two chunks of 32 query columns
-        const uint32_t col = hq * 64 + c * 32;
-        uint32_t sv[32], dv[32], pp[16], zz[16];
-        tmem_ld32(tmem + lane_off + col, sv);
-        tmem_ld32(tmem + 128 + lane_off + col, dv);
+        uint32_t sv[32], pp[16];
+        tmem_ld32(tmem + lane_off + hq * 64 + c * 32, sv);
         tmem_wait_ld();
         if (mode == kMasked) {
 #pragma unroll
-          for (int k = 0; k < 16; ++k) pp[k] = zz[k] = 0u;
+          for (int k = 0; k < 32; ++k) pr[c * 32 + k] = 0.f;
         } else {
 #pragma unroll
           for (int k = 0; k < 32; k += 4) {
             const float4 l4 = *reinterpret_cast<const float4*>(lse_s + c * 32 + k);
-            const float4 d4 = *reinterpret_cast<const float4*>(dvec_s + c * 32 + k);
 #pragma unroll
             for (int e = 0; e < 4; e += 2) {
               const int i = k + e;
-              // x = scale*log2e*s + bias*log2e - LSE*log2e, two columns at a time
               f32x2 x2 = f2_fma(f2_make(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), scv, biasv);
               x2 = f2_fma(e == 0 ? f2_make(l4.x, l4.y) : f2_make(l4.z, l4.w), nlog2e, x2);
               float x0, x1;
@@ -348,22 +370,51 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 if (c * 32 + i < jloc) x0 = -INFINITY;
                 if (c * 32 + i + 1 < jloc) x1 = -INFINITY;
               }
-              const float p0 = ex2(x0), p1 = ex2(x1);
+              pr[c * 32 + i] = ex2(x0);
+              pr[c * 32 + i + 1] = ex2(x1);
+            }
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 16; ++k) pp[k] = pack_bf16(pr[c * 32 + 2 * k], pr[c * 32 + 2 * k + 1]);
+        // bf16 P^T stays inside this warp's own 64 S^T columns, over ones already read
+        tmem_st16(tmem + lane_off + hq * 64 + c * 16, pp);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->pa_full);
+      // phase B: dZ^T = P^T o (dP^T - D)
+      if (!mbar_wait(&bars->dp_full, j & 1, abort_flag, a.err, kTimeoutNs)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      f32x2 g2 = f2_make(0.f, 0.f);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t dv[32], zz[16];
+        tmem_ld32(tmem + 128 + lane_off + hq * 64 + c * 32, dv);
+        tmem_wait_ld();
+        if (mode == kMasked) {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) zz[k] = 0u;
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; k += 4) {
+            const float4 d4 = *reinterpret_cast<const float4*>(dvec_s + c * 32 + k);
+#pragma unroll
+            for (int e = 0; e < 4; e += 2) {
+              const int i = k + e;
               const f32x2 dd = f2_sub(f2_make(__uint_as_float(dv[i]), __uint_as_float(dv[i + 1])),
                                       e == 0 ? f2_make(d4.x, d4.y) : f2_make(d4.z, d4.w));
-              const f32x2 dz = f2_mul(f2_make(p0, p1), dd);
+              const f32x2 dz = f2_mul(f2_make(pr[c * 32 + i], pr[c * 32 + i + 1]), dd);
               g2 = f2_add(g2, dz);
               float dz0, dz1;
               f2_split(dz, dz0, dz1);
-              pp[i / 2] = pack_bf16(p0, p1);
               zz[i / 2] = pack_bf16(dz0, dz1);
             }
           }
         }
-        // packed outputs stay inside this warp's own 64 columns of S^T / dP^T
-        // (which the other warp of the quadrant never reads), over columns
-        // already consumed by this chunk
-        tmem_st16(tmem + lane_off + hq * 64 + c * 16, pp);
         tmem_st16(tmem + 128 + lane_off + hq * 64 + c * 16, zz);
 #pragma unroll
         for (int gi = 0; gi < 4; ++gi) {
@@ -372,17 +423,16 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
               make_uint4(zz[4 * gi], zz[4 * gi + 1], zz[4 * gi + 2], zz[4 * gi + 3]);
         }
       }
-      float g, g_hi;
-      f2_split(g2, g, g_hi);
-      g += g_hi;
-      g = warp_sum(g);
-      if (lane == 0 && mode != kMasked) atomicAdd(a.Gblk + ((size_t)bh * p.Nb + r) * p.Nb + cj, g);
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars->p_full);
+      mbar_arrive(&bars->pb_full);
+      float g, g_hi;
+      f2_split(g2, g, g_hi);
+      g = warp_sum(g + g_hi);
+      if (lane == 0 && mode != kMasked) atomicAdd(a.Gblk + ((size_t)bh * p.Nb + r) * p.Nb + cj, g);
 
-      // drain dQ (TMEM lane == query row) into the fp32 accumulator
+      // drain dQ (in R1; TMEM lane == query row) into the fp32 accumulator
       if (!mbar_wait(&bars->dq_full, j & 1, abort_flag, a.err, kTimeoutNs)) {
         ok = false;
         break;
@@ -395,7 +445,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 #pragma unroll
       for (int bx = 0; bx < D / 64; ++bx) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_off + hq * (D / 2) + bx * 32, o);
+        tmem_ld32(tmem + 128 + lane_off + hq * (D / 2) + bx * 32, o);
         tmem_wait_ld();
         uint8_t* row = stg + bx * 4096 + lane * 128;
 #pragma unroll
@@ -405,7 +455,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars->dq_free);  // TMEM is free; the reduction proceeds from smem
+      mbar_arrive(&bars->dq_free);  // R1 is free; the reduction proceeds from smem
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->staged[st]);  // the producer issues the reduction
     }
