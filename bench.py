@@ -204,8 +204,8 @@ def bench_training(w, steps, warmup, rank, dev, peaks):
     fl_fwd, fl_fb = 4.0 * w.d * P, 14.0 * w.d * P
     ms = statistics.mean(step_ms)
     kern = {
-        "fwd_tc_kernel": {"ms": statistics.mean(fwd_ms), "flops": fl_fwd},
-        "bwd_main": {"ms": statistics.mean(bwd_ms), "flops": fl_fb - fl_fwd},
+        "fwd_tc2_kernel": {"ms": statistics.mean(fwd_ms), "flops": fl_fwd},
+        "bwd_tc_kernel": {"ms": statistics.mean(bwd_ms), "flops": fl_fb - fl_fwd},
     }
     dom = max(kern, key=lambda n: kern[n]["ms"])
     ach = kern[dom]["flops"] / (kern[dom]["ms"] * 1e-3) / 1e12
