@@ -482,6 +482,14 @@ cudaError_t launch_typed(const FwdArgs& a, const void* Q, const void* K, const v
 
 }  // namespace
 
+cudaError_t launch_plan(const Problem& p, const Selection& sel, int32_t* plan, int plan_stride,
+                        int n_tiles, cudaStream_t st) {
+  const int n = p.B * p.Hq * n_tiles;
+  plan_kernel<<<(n + 127) / 128, 128, 0, st>>>(p, sel, plan, plan_stride, n_tiles);
+  note_launch();
+  return cudaGetLastError();
+}
+
 bool fwd_tc_supported(const Problem& p) {
   return p.dtype == GBS_BF16 && p.bs == kSlot && (p.d == 64 || p.d == 128) && p.N % kSlot == 0;
 }

@@ -65,6 +65,16 @@ cudaError_t launch_fwd_tc2(const Problem& p, const void* Q, const void* K, const
                            const float* S, const float* slse, void* O, float* LSE,
                            unsigned int* err, cudaStream_t st);
 bool fwd_tc2_supported(const Problem& p);
+// Per-(batch, head, 128-row tile) slot plan of sparse mode (union of the tile's
+// two query blocks' Top-K lists plus their current blocks, with per-half biases).
+cudaError_t launch_plan(const Problem& p, const Selection& sel, int32_t* plan, int plan_stride,
+                        int n_tiles, cudaStream_t st);
+// Sparse mode, even q-heads-per-kv-head ratio: two query tiles per CTA, one
+// context block per pipeline stage.
+cudaError_t launch_fwd_sp(const Problem& p, const void* Q, const void* K, const void* V,
+                          const Selection& sel, int32_t* plan, int plan_stride, void* O,
+                          float* LSE, unsigned int* err, cudaStream_t st);
+bool fwd_sp_supported(const Problem& p);
 cudaError_t launch_bwd_tc(const Problem& p, const void* Q, const void* K, const void* V,
                           const float* S, const float* slse, const void* O, const float* LSE,
                           const void* dO, void* dQ, void* dK, void* dV, float* Dvec, float* Gblk,

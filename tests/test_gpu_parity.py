@@ -137,6 +137,30 @@ def test_fwd_edge_shapes(shape, mode, k):
         _check_fwd(x, mode, k, tol)
 
 
+@pytest.mark.parametrize("shape,k", [
+    ((1, 4, 2, 320, 128), 2),    # odd block count, two q-heads per kv-head pair
+    ((2, 8, 2, 448, 64), 3),     # d = 64, G = 4
+    ((1, 4, 2, 512, 128), 0),    # current block only
+    ((1, 4, 2, 512, 128), 100),  # full budget: equals training mode
+    ((1, 8, 4, 1024, 128), 5),
+])
+@pytest.mark.parametrize("scaled", [True, False])
+def test_fwd_sparse_two_tile_kernel(shape, k, scaled):
+    """Sparse mode with an even q-heads-per-kv-head ratio (two tiles per CTA)."""
+    B, Hq, Hkv, N, d = shape
+    x = _small(23 + k, B, Hq, Hkv, N, d, torch.bfloat16, scaled)
+    _check_fwd(x, "sparse", k, TOL_BF16)
+
+
+def test_fwd_sparse_full_budget_matches_training():
+    x = _small(29, 1, 4, 2, 512, 128, torch.bfloat16, False)
+    Qd, Kd, Vd, Sd = (x[n].to(DEV) for n in "QKVS")
+    Ot, Lt = gb.forward(Qd, Kd, Vd, Sd, mode="train")
+    Os, Ls = gb.forward(Qd, Kd, Vd, Sd, mode="sparse", topk=8)
+    torch.cuda.synchronize()
+    assert rel_err(np64(Os), np64(Ot)) < 1e-2 and rel_err(Ls.cpu().numpy(), Lt.cpu().numpy()) < 1e-5
+
+
 def test_fwd_train_full_size_sampled():
     """Training workload N=8192, 32/8 heads, bf16: sampled query blocks."""
     w = WORKLOADS["train_bf16_n8192"]
