@@ -7,13 +7,15 @@
 // Abstract).
 //
 // One warp owns one score row. Training mode only needs the row's log-sum-exp
-// over the historical blocks c < r. Sparse mode finds the K-th largest score by
-// a most-significant-bit-first threshold search on order-preserving 32-bit
-// keys (32 counting passes over the row in shared memory), keeps every block
-// above the threshold plus the lowest-index blocks equal to it, compacts them
-// in ascending index order with ballots, and renormalises the log gates over
-// the kept set. Comparisons are exact on the fp32 scores, so the index lists
-// are bit-identical to any other exact implementation of the same ordering.
+// over the historical blocks c < r. Sparse mode maps the scores to
+// order-preserving 32-bit keys once (in shared memory), finds the K-th largest
+// key by an 8-bit radix select (four histogram passes, most significant digit
+// first, per-warp bins, a warp scan to locate the bin holding rank K), keeps
+// every block above that key plus the lowest-index blocks equal to it,
+// compacts them in ascending index order with ballots, and renormalises the
+// log gates over the kept set. Comparisons are exact on the fp32 scores, so
+// the index lists are bit-identical to any other exact implementation of the
+// same ordering.
 #include "common.cuh"
 #include "internal.h"
 
@@ -29,11 +31,49 @@ __device__ __forceinline__ float row_score(const float* srow, const uint32_t* ca
   return cached ? __uint_as_float(cache[c]) : __ldg(srow + c);
 }
 
+// Locates, among the 256 bins of `hist` (lane l holds bins 8l..8l+7), the bin
+// holding the element of rank kk counted from the top, and the number of
+// elements in higher bins.
+__device__ __forceinline__ int find_bin(const uint32_t* hist, int kk, int lane, int* above_out) {
+  int c[8];
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    c[i] = (int)hist[8 * lane + i];
+    sum += c[i];
+  }
+  int incl = sum;  // sum over lanes >= lane
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_down_sync(0xffffffffu, incl, o);
+    if (lane + o < 32) incl += t;
+  }
+  const int excl = incl - sum;  // sum over lanes > lane (higher bins)
+  const unsigned bal = __ballot_sync(0xffffffffu, excl < kk && kk <= incl);
+  const int src = __ffs(bal) - 1;
+  int bin = 0, above = 0;
+  if (lane == src) {
+    int acc = excl;
+    for (int i = 7; i >= 0; --i) {
+      if (acc + c[i] >= kk) {
+        bin = 8 * lane + i;
+        above = acc;
+        break;
+      }
+      acc += c[i];
+    }
+  }
+  bin = __shfl_sync(0xffffffffu, bin, src);
+  *above_out = __shfl_sync(0xffffffffu, above, src);
+  return bin;
+}
+
 __global__ void __launch_bounds__(kWarps * 32)
 select_kernel(const float* __restrict__ S, int n_rows, int row_stride, int rows_per_head,
               int decode_cur, int topk, int sparse, int32_t* __restrict__ idx,
               int32_t* __restrict__ cnt, float* __restrict__ logg, float* __restrict__ slse) {
   __shared__ uint32_t cache_all[kWarps][kRowCache];
+  __shared__ uint32_t hist_all[kWarps][256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * kWarps + warp;
   if (row >= n_rows) return;
@@ -61,10 +101,43 @@ select_kernel(const float* __restrict__ S, int n_rows, int row_stride, int rows_
   int32_t* out_idx = idx + (size_t)row * topk;
   float* out_logg = logg + (size_t)row * topk;
 
-  // Threshold T = the k-th largest key; count_ge(T) >= k and count_gt(T) < k.
+  // Threshold T = the k-th largest key; need_eq = how many keys equal to T
+  // (lowest indices first) complete the top k.
   uint32_t T = 0u;
   int need_eq = 0;
-  if (k > 0 && k < r) {
+  if (k > 0 && k < r && cached) {
+    // keys once, then four 8-bit digit passes
+    for (int c = lane; c < r; c += 32) cache[c] = ordered_key(__uint_as_float(cache[c]));
+    __syncwarp();
+    uint32_t* hist = hist_all[warp];
+    uint32_t prefix = 0u, mask = 0u;
+    int kk = k;
+#pragma unroll 1
+    for (int shift = 24; shift >= 0; shift -= 8) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) hist[8 * lane + i] = 0u;
+      __syncwarp();
+      for (int c = lane; c < r; c += 32) {
+        const uint32_t u = cache[c];
+        if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+      }
+      __syncwarp();
+      int above;
+      const int bin = find_bin(hist, kk, lane, &above);
+      kk -= above;
+      prefix |= (uint32_t)bin << shift;
+      mask |= 255u << shift;
+      __syncwarp();
+    }
+    T = prefix;
+    need_eq = kk;
+    // back to scores for the compaction and the gate normalisation below
+    for (int c = lane; c < r; c += 32) {
+      const uint32_t u = cache[c];
+      cache[c] = (u & 0x80000000u) ? (u & 0x7fffffffu) : ~u;
+    }
+    __syncwarp();
+  } else if (k > 0 && k < r) {
     for (int bit = 31; bit >= 0; --bit) {
       const uint32_t cand = T | (1u << bit);
       int n = 0;
