@@ -32,7 +32,9 @@
 // The next step's S^T is issued as soon as dQ is issued, so its phase A
 // overlaps the drain of dQ and the dP^T MMA.
 // Warps: 0-7 compute (lane quadrant w%4, query/column half w/4), 8 TMA,
-// 9 TMEM allocator + MMA issuer. Every mbarrier wait is bounded.
+// 9 TMEM allocator + MMA issuer, 10-13 dQ drain (lane quadrant w%4): the
+// drain warps move dQ out of TMEM while the compute warps start the next
+// step. Every mbarrier wait is bounded.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -49,7 +51,9 @@ constexpr int kBK = 128;         // keys per CTA
 constexpr int kBQ = 128;         // queries per step
 constexpr int kQStages = 2;
 constexpr int kComputeWarps = 8;
-constexpr int kThreads = (kComputeWarps + 2) * 32;
+constexpr int kDrainWarps = 4;  // one per TMEM lane quadrant
+constexpr int kTmaWarp = kComputeWarps, kMmaWarp = kComputeWarps + 1;
+constexpr int kThreads = (kComputeWarps + 2 + kDrainWarps) * 32;
 constexpr int kTmemCols = 512;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 constexpr int kChunk = 128 * 128;  // bytes of one 64-column chunk of a 128-row tile
@@ -71,7 +75,7 @@ struct BLayout {
 struct BBarriers {
   uint64_t kv_full;
   uint64_t q_full[kQStages];
-  uint64_t staged[kQStages];  // every compute warp has staged the step's dQ in this stage
+  uint64_t staged[kQStages];  // every drain warp has staged the step's dQ in this stage
   uint64_t s_full;   // S^T of the step landed in R0
   uint64_t dp_full;  // dP^T of the step landed in R1
   uint64_t pa_full;  // P^T written (dV can start)
@@ -136,19 +140,19 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     mbar_init(&bars->kv_full, 1);
     for (int s = 0; s < kQStages; ++s) {
       mbar_init(&bars->q_full[s], 1);
-      mbar_init(&bars->staged[s], kComputeWarps);
+      mbar_init(&bars->staged[s], kDrainWarps);
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->dp_full, 1);
     mbar_init(&bars->pa_full, kComputeWarps * 32);
     mbar_init(&bars->pb_full, kComputeWarps * 32);
     mbar_init(&bars->dq_full, 1);
-    mbar_init(&bars->dq_free, kComputeWarps * 32);
+    mbar_init(&bars->dq_free, kDrainWarps * 32);
     mbar_init(&bars->done, 1);
     bars->abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -159,7 +163,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   volatile int* abort_flag = &bars->abort_flag;
   float* vecs = reinterpret_cast<float*>(smem + L::kVecOff);
 
-  if (warp == 8) {
+  if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tmQ);
@@ -234,7 +238,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           mbar_wait(&bars->q_full[j % kQStages], (j / kQStages) & 1, abort_flag, nullptr, 1000000ull);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     // -------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idST = idesc_bf16_f32(kBK, kBQ, 0, 0);  // S^T, dP^T
@@ -311,7 +315,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       mma_commit(&bars->done);
       mbar_wait(&bars->done, 0, abort_flag, a.err, kTimeoutNs);
     }
-  } else {
+  } else if (warp < kComputeWarps) {
     // ------------------------------------------------------- compute warps
     const int quad = warp & 3, hq = warp >> 2;
     const int krow = quad * 32 + lane;  // key row within the tile == TMEM lane
@@ -391,23 +395,23 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       tc_fence_after();
       f32x2 g2 = f2_make(0.f, 0.f);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t dv[32], zz[16];
-        tmem_ld32(tmem + 128 + lane_off + hq * 64 + c * 32, dv);
+      for (int c = 0; c < 4; ++c) {  // four chunks of 16 query columns
+        uint32_t dv[16], zz[8];
+        tmem_ld16(tmem + 128 + lane_off + hq * 64 + c * 16, dv);
         tmem_wait_ld();
         if (mode == kMasked) {
 #pragma unroll
-          for (int k = 0; k < 16; ++k) zz[k] = 0u;
+          for (int k = 0; k < 8; ++k) zz[k] = 0u;
         } else {
 #pragma unroll
-          for (int k = 0; k < 32; k += 4) {
-            const float4 d4 = *reinterpret_cast<const float4*>(dvec_s + c * 32 + k);
+          for (int k = 0; k < 16; k += 4) {
+            const float4 d4 = *reinterpret_cast<const float4*>(dvec_s + c * 16 + k);
 #pragma unroll
             for (int e = 0; e < 4; e += 2) {
               const int i = k + e;
               const f32x2 dd = f2_sub(f2_make(__uint_as_float(dv[i]), __uint_as_float(dv[i + 1])),
                                       e == 0 ? f2_make(d4.x, d4.y) : f2_make(d4.z, d4.w));
-              const f32x2 dz = f2_mul(f2_make(pr[c * 32 + i], pr[c * 32 + i + 1]), dd);
+              const f32x2 dz = f2_mul(f2_make(pr[c * 16 + i], pr[c * 16 + i + 1]), dd);
               g2 = f2_add(g2, dz);
               float dz0, dz1;
               f2_split(dz, dz0, dz1);
@@ -415,10 +419,12 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
           }
         }
-        tmem_st16(tmem + 128 + lane_off + hq * 64 + c * 16, zz);
+        // dZ^T of keys' query columns [16 c, 16 c + 16) -> packed columns [8 c, 8 c + 8)
+        // of this warp's 64 dP^T columns, all already read by chunks 0..c
+        tmem_st8(tmem + 128 + lane_off + hq * 64 + c * 8, zz);
 #pragma unroll
-        for (int gi = 0; gi < 4; ++gi) {
-          const int gg = c * 4 + gi;
+        for (int gi = 0; gi < 2; ++gi) {
+          const int gg = c * 2 + gi;
           *reinterpret_cast<uint4*>(zrow + ((gg ^ (krow & 7)) << 4)) =
               make_uint4(zz[4 * gi], zz[4 * gi + 1], zz[4 * gi + 2], zz[4 * gi + 3]);
         }
@@ -431,34 +437,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       f2_split(g2, g, g_hi);
       g = warp_sum(g + g_hi);
       if (lane == 0 && mode != kMasked) atomicAdd(a.Gblk + ((size_t)bh * p.Nb + r) * p.Nb + cj, g);
-
-      // drain dQ (in R1; TMEM lane == query row) into the fp32 accumulator
-      if (!mbar_wait(&bars->dq_full, j & 1, abort_flag, a.err, kTimeoutNs)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // stage this warp's 32 rows x D/2 columns of dQ (128-byte swizzled boxes
-      // of 32 x 32 fp32) in the step's Q (hq 0) or dO (hq 1) stage, which every
-      // MMA of the step has finished reading
-      uint8_t* stg = smem + (hq == 0 ? L::kQOff : L::kdOOff) + st * L::kTile + quad * (D / 2) * 128;
-#pragma unroll
-      for (int bx = 0; bx < D / 64; ++bx) {
-        uint32_t o[32];
-        tmem_ld32(tmem + 128 + lane_off + hq * (D / 2) + bx * 32, o);
-        tmem_wait_ld();
-        uint8_t* row = stg + bx * 4096 + lane * 128;
-#pragma unroll
-        for (int gi = 0; gi < 8; ++gi)
-          *reinterpret_cast<uint4*>(row + ((gi ^ (lane & 7)) << 4)) =
-              make_uint4(o[4 * gi], o[4 * gi + 1], o[4 * gi + 2], o[4 * gi + 3]);
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&bars->dq_free);  // R1 is free; the reduction proceeds from smem
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->staged[st]);  // the producer issues the reduction
     }
+
     // epilogue: dV and dK rows of this tile (TMEM lane == key row)
     if (ok && mbar_wait(&bars->done, 0, abort_flag, a.err, kTimeoutNs)) {
       tc_fence_after();
@@ -490,10 +470,40 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
       }
     }
+  } else {
+    // ------------------------------------------------------- dQ drain warps
+    const int quad = warp & 3;  // TMEM lane quadrant == 32 query rows of dQ
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    for (int j = 0; j < n_steps; ++j) {
+      const int st = j % kQStages;
+      if (!mbar_wait(&bars->dq_full, j & 1, abort_flag, a.err, kTimeoutNs)) break;
+      tc_fence_after();
+      // 32 rows x D columns as 32 x 32 fp32 boxes (128-byte swizzle): columns
+      // [0, D/2) go to the step's Q stage, [D/2, D) to its dO stage; every MMA
+      // of the step has finished reading both
+#pragma unroll
+      for (int bx = 0; bx < D / 32; ++bx) {
+        const int hq = bx / (D / 64), sub = bx % (D / 64);
+        uint8_t* row = smem + (hq == 0 ? L::kQOff : L::kdOOff) + st * L::kTile +
+                       quad * (D / 2) * 128 + sub * 4096 + lane * 128;
+        uint32_t o[32];
+        tmem_ld32(tmem + 128 + lane_off + bx * 32, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int gi = 0; gi < 8; ++gi)
+          *reinterpret_cast<uint4*>(row + ((gi ^ (lane & 7)) << 4)) =
+              make_uint4(o[4 * gi], o[4 * gi + 1], o[4 * gi + 2], o[4 * gi + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars->dq_free);  // R1 is free; the reduction proceeds from smem
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->staged[st]);  // the TMA warp issues the reduction
+    }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
