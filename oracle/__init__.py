@@ -6,6 +6,7 @@ imports it and it never imports the CUDA library.
 """
 from .gated_attention import (  # noqa: F401
     SPARSE,
+    THRESHOLD,
     TRAIN,
     attended_blocks,
     attended_pairs,
@@ -15,4 +16,5 @@ from .gated_attention import (  # noqa: F401
     gated_decode,
     log_gates,
     select_blocks,
+    threshold_count,
 )

@@ -58,6 +58,7 @@ import numpy as np
 
 TRAIN = "train"
 SPARSE = "sparse"
+THRESHOLD = "threshold"
 
 
 def _as_f64(x):
@@ -70,22 +71,42 @@ def _logsumexp(x):
     return m + np.log(np.sum(np.exp(x - m)))
 
 
-def attended_blocks(s_row, r, mode, topk):
+def threshold_count(s_row, r, tau):
+    """Number of blocks c < r whose training-mode gate g[r, c] is at least tau.
+
+    The dynamic threshold of the viyan blog ("Implementation and Efficiency":
+    only blocks above a threshold are computed) read on the normalised gate:
+    S[r, c] - logsumexp(S[r, :r]) >= ln tau.
+    """
+    if r == 0:
+        return 0
+    s = _as_f64(s_row[:r])
+    return int(np.sum(s - _logsumexp(s) >= np.log(tau)))
+
+
+def attended_blocks(s_row, r, mode, topk, tau=None):
     """The historical set A_r of query block r (ascending block indices).
 
     Training mode keeps every earlier block (poster Abstract: all context units
     stay active during training). Sparse mode keeps a fixed budget of min(K, r)
     earlier blocks with the largest scores (poster Abstract: fixed attention
-    budget; HF page Abstract: hard Top-K). Ordering is score descending, then
-    block index ascending; -0.0 and +0.0 compare equal.
+    budget; HF page Abstract: hard Top-K). Threshold mode keeps the blocks whose
+    gate reaches tau, at most K of them (the largest scores first); since the
+    passing blocks are exactly the highest-scoring ones, it is Top-K with
+    K = min(topk, threshold_count). Ordering is score descending, then block
+    index ascending; -0.0 and +0.0 compare equal.
     """
     if mode == TRAIN:
         return np.arange(r, dtype=np.int64)
-    if mode != SPARSE:
+    if mode not in (SPARSE, THRESHOLD):
         raise ValueError(f"unknown mode {mode!r}")
     if topk is None or topk < 0:
-        raise ValueError("sparse mode needs topk >= 0")
+        raise ValueError("sparse and threshold modes need topk >= 0")
     k = min(int(topk), r)
+    if mode == THRESHOLD:
+        if tau is None or not (0.0 < tau <= 1.0):
+            raise ValueError("threshold mode needs 0 < tau <= 1")
+        k = min(k, threshold_count(s_row, r, tau))
     if k == 0:
         return np.zeros(0, dtype=np.int64)
     s = _as_f64(s_row[:r])
@@ -114,10 +135,10 @@ def log_gates(s_row, A, r, renormalise=True, gate="log_softmax"):
     return s[A] - _logsumexp(s[norm_set])
 
 
-def _query_block(Q, K, V, S, b, h, r, bs, N, G, mode, topk, scale, renormalise, gate):
+def _query_block(Q, K, V, S, b, h, r, bs, N, G, mode, topk, scale, renormalise, gate, tau=None):
     """Keys, values, logits and bookkeeping of one (batch, q-head, query block)."""
     i0, i1 = r * bs, min((r + 1) * bs, N)
-    A = attended_blocks(S[b, h, r], r, mode, topk)
+    A = attended_blocks(S[b, h, r], r, mode, topk, tau)
     lg = log_gates(S[b, h, r], A, r, renormalise, gate)
     kv = h // G
     cols = [np.arange(c * bs, (c + 1) * bs) for c in A]
@@ -159,7 +180,7 @@ def _check_shapes(Q, K, V, S, bs):
 
 
 def gated_attention_forward(Q, K, V, S, block, mode=TRAIN, topk=None, scale=None,
-                            renormalise=True, gate="log_softmax", rows=None):
+                            renormalise=True, gate="log_softmax", rows=None, tau=None):
     """Forward pass, blockwise: returns (O, LSE) in float64.
 
     Never forms the N x N matrix; each query block gathers the keys of
@@ -177,7 +198,7 @@ def gated_attention_forward(Q, K, V, S, block, mode=TRAIN, topk=None, scale=None
     todo = rows if rows is not None else [(b, h, r) for b in range(B) for h in range(Hq) for r in range(Nb)]
     for b, h, r in todo:
         *_, v, z, (i0, i1), _ = _query_block(Q, K, V, S, b, h, r, block, N, G, mode, topk,
-                                             scale, renormalise, gate)
+                                             scale, renormalise, gate, tau)
         p, lse = _softmax_rows(z)
         O[b, h, i0:i1] = p @ v
         LSE[b, h, i0:i1] = lse
@@ -185,7 +206,7 @@ def gated_attention_forward(Q, K, V, S, block, mode=TRAIN, topk=None, scale=None
 
 
 def gated_attention_backward(Q, K, V, S, dO, block, mode=TRAIN, topk=None, scale=None,
-                             renormalise=True, gate="log_softmax", heads=None):
+                             renormalise=True, gate="log_softmax", heads=None, tau=None):
     """Backward pass: returns (dQ, dK, dV, dS, Gsum) in float64.
 
     The gradient reaches the scores because they sit inside the softmax
@@ -213,7 +234,7 @@ def gated_attention_backward(Q, K, V, S, dO, block, mode=TRAIN, topk=None, scale
             Gsum[b, h] = 0.0
             for r in range(Nb):
                 A, lg, cols, q, k, v, z, (i0, i1), kv = _query_block(
-                    Q, K, V, S, b, h, r, block, N, G, mode, topk, scale, renormalise, gate)
+                    Q, K, V, S, b, h, r, block, N, G, mode, topk, scale, renormalise, gate, tau)
                 p, _ = _softmax_rows(z)
                 do = _as_f64(dO[b, h, i0:i1])
                 dp = do @ v.T
@@ -240,7 +261,7 @@ def gated_attention_backward(Q, K, V, S, dO, block, mode=TRAIN, topk=None, scale
 
 
 def gated_attention_naive(Q, K, V, S, block, mode=TRAIN, topk=None, scale=None,
-                          renormalise=True, gate="log_softmax"):
+                          renormalise=True, gate="log_softmax", tau=None):
     """Forward pass with the full N x N logit matrix per head (tiny inputs only).
 
     Returns (O, LSE, bias) with the token-level bias matrix [B, Hq, N, N].
@@ -256,7 +277,7 @@ def gated_attention_naive(Q, K, V, S, block, mode=TRAIN, topk=None, scale=None,
         for h in range(Hq):
             for i in range(N):
                 r = i // block
-                A = attended_blocks(S[b, h, r], r, mode, topk)
+                A = attended_blocks(S[b, h, r], r, mode, topk, tau)
                 lg = log_gates(S[b, h, r], A, r, renormalise, gate)
                 for a, c in enumerate(A):
                     bias[b, h, i, c * block:(c + 1) * block] = lg[a]
@@ -269,7 +290,7 @@ def gated_attention_naive(Q, K, V, S, block, mode=TRAIN, topk=None, scale=None,
     return O, LSE, bias
 
 
-def select_blocks(S, block_count, topk, mode=SPARSE):
+def select_blocks(S, block_count, topk, mode=SPARSE, tau=None):
     """Index-list form of A_r for every (b, h, r): (idx, cnt, logg, slse).
 
     idx [B, H, Nb, K] int32 ascending, padded with -1; cnt [B, H, Nb] int32;
@@ -288,7 +309,7 @@ def select_blocks(S, block_count, topk, mode=SPARSE):
     for b in range(B):
         for h in range(H):
             for r in range(Nb):
-                A = attended_blocks(S[b, h, r], r, mode, K)
+                A = attended_blocks(S[b, h, r], r, mode, K, tau)
                 cnt[b, h, r] = len(A)
                 idx[b, h, r, :len(A)] = A
                 logg[b, h, r, :len(A)] = log_gates(S[b, h, r], A, r)
@@ -297,7 +318,8 @@ def select_blocks(S, block_count, topk, mode=SPARSE):
     return idx, cnt, logg, slse
 
 
-def gated_decode(q, Kc, Vc, S_dec, L, block, topk, scale=None, seqs=None, gate="log_softmax"):
+def gated_decode(q, Kc, Vc, S_dec, L, block, topk, scale=None, seqs=None, gate="log_softmax",
+                 mode=SPARSE, tau=None):
     """Sparse decode of one query per sequence: returns (O [B,Hq,d], LSE [B,Hq]).
 
     The query sits at position L-1 (HF page Abstract: the current block is
@@ -317,7 +339,7 @@ def gated_decode(q, Kc, Vc, S_dec, L, block, topk, scale=None, seqs=None, gate="
     LSE = np.full((B, Hq), np.nan)
     for b in (seqs if seqs is not None else range(B)):
         for h in range(Hq):
-            A = attended_blocks(S_dec[b, h], cur, SPARSE, topk)
+            A = attended_blocks(S_dec[b, h], cur, mode, topk, tau)
             lg = log_gates(S_dec[b, h], A, cur, True, gate)
             cols = [np.arange(c * block, (c + 1) * block) for c in A]
             cols.append(np.arange(cur * block, L))
@@ -334,7 +356,7 @@ def gated_decode(q, Kc, Vc, S_dec, L, block, topk, scale=None, seqs=None, gate="
     return O, LSE
 
 
-def attended_pairs(S, N, block, mode=TRAIN, topk=None):
+def attended_pairs(S, N, block, mode=TRAIN, topk=None, tau=None):
     """Number of attended (i, j) pairs per (b, h): the FLOP-count basis.
 
     A historical block contributes bs*bs pairs; the current block the causal
@@ -347,7 +369,7 @@ def attended_pairs(S, N, block, mode=TRAIN, topk=None):
             tot = 0
             for r in range(Nb):
                 rows = min(N, (r + 1) * block) - r * block
-                A = attended_blocks(S[b, h, r], r, mode, topk)
+                A = attended_blocks(S[b, h, r], r, mode, topk, tau)
                 tot += len(A) * block * rows + rows * (rows + 1) // 2
             out[b, h] = tot
     return out

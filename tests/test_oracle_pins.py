@@ -260,6 +260,54 @@ def test_negative_zero_equals_positive_zero():
     assert list(oracle.attended_blocks(s2, 3, oracle.SPARSE, 1)) == [0]
 
 
+# ------------------------------------------------------------ dynamic threshold
+
+def _brute_threshold(s, r, k, tau):
+    """Blocks whose gate exp(s_c - logsumexp(s)) reaches tau, keeping the k best."""
+    if r == 0:
+        return []
+    g = np.exp(s[:r] - np.log(np.sum(np.exp(s[:r]))))
+    passing = [c for c in range(r) if g[c] >= tau]
+    passing.sort(key=lambda c: (-s[c], c))
+    return sorted(passing[:k])
+
+
+def test_threshold_selection_against_definition():
+    rng = np.random.default_rng(31)
+    for trial in range(60):
+        r = int(rng.integers(0, 30))
+        s = rng.standard_normal(r) * math.sqrt(2)
+        for tau in (1e-4, 0.02, 0.1, 0.3, 1.0):
+            for k in (0, 2, 5, 40):
+                got = list(oracle.attended_blocks(s, r, oracle.THRESHOLD, k, tau))
+                assert got == _brute_threshold(s, r, k, tau), (trial, tau, k)
+
+
+def test_threshold_limits():
+    """tau below every gate with an unlimited budget is training mode; tau = 1
+    keeps a block only when it is the sole historical block."""
+    Q, K, V, S, _ = _rand(32, 1, 2, 1, 96, 8, 16)
+    O1, L1 = oracle.gated_attention_forward(Q, K, V, S, 16)
+    O2, L2 = oracle.gated_attention_forward(Q, K, V, S, 16, mode=oracle.THRESHOLD, topk=100, tau=1e-30)
+    assert np.array_equal(O1, O2) and np.array_equal(L1, L2)
+    idx, cnt, _, _ = oracle.select_blocks(S, 6, 100, mode=oracle.THRESHOLD, tau=1.0)
+    assert list(cnt[0, 0]) == [0, 1, 0, 0, 0, 0]
+
+
+def test_threshold_is_topk_with_passing_count():
+    S = np.random.default_rng(33).standard_normal((1, 2, 20, 20)) * math.sqrt(2)
+    for tau in (0.05, 0.15):
+        for k in (3, 8):
+            it, ct, lt, _ = oracle.select_blocks(S, 20, k, mode=oracle.THRESHOLD, tau=tau)
+            for h in range(2):
+                for r in range(20):
+                    kk = min(k, oracle.threshold_count(S[0, h, r], r, tau))
+                    ref = oracle.attended_blocks(S[0, h, r], r, oracle.SPARSE, kk)
+                    assert ct[0, h, r] == len(ref) and list(it[0, h, r, :len(ref)]) == list(ref)
+                    if len(ref):
+                        assert abs(np.exp(lt[0, h, r, :len(ref)]).sum() - 1) < 1e-14
+
+
 # ----------------------------------------------------------------------- decode
 
 @pytest.mark.parametrize("L", [64, 80, 127])
