@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(HERE, "libgbs.so")
 GBS_OK = 0
 STATUS_NAMES = {0: "GBS_OK", 1: "GBS_ERR_INVALID_ARG", 2: "GBS_ERR_UNSUPPORTED", 3: "GBS_ERR_CUDA",
                 4: "GBS_ERR_TIMEOUT", 5: "GBS_ERR_WORKSPACE"}
-MODES = {"train": 0, "sparse": 1}
+MODES = {"train": 0, "sparse": 1, "threshold": 2}
 DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 OP_FWD, OP_BWD, OP_DECODE = 0, 1, 2
 
@@ -36,7 +36,7 @@ class Params(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
                 ("N", ctypes.c_int), ("d", ctypes.c_int), ("block", ctypes.c_int),
                 ("topk", ctypes.c_int), ("mode", ctypes.c_int), ("dtype", ctypes.c_int),
-                ("scale", ctypes.c_float)]
+                ("scale", ctypes.c_float), ("tau", ctypes.c_float)]
 
 
 _lib = None
@@ -89,8 +89,10 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def make_params(B, Hq, Hkv, N, d, block=64, topk=0, mode="train", dtype=torch.bfloat16, scale=0.0):
-    return Params(B, Hq, Hkv, N, d, block, topk, MODES[mode], DTYPES[dtype], float(scale))
+def make_params(B, Hq, Hkv, N, d, block=64, topk=0, mode="train", dtype=torch.bfloat16, scale=0.0,
+                tau=0.0):
+    return Params(B, Hq, Hkv, N, d, block, topk, MODES[mode], DTYPES[dtype], float(scale),
+                  float(tau))
 
 
 def workspace_bytes(params: Params, op: int) -> int:
@@ -106,20 +108,20 @@ def alloc_workspace(params: Params, op: int, device) -> torch.Tensor:
     return ws
 
 
-def _prefill_params(Q, K, S, block, topk, mode, scale):
+def _prefill_params(Q, K, S, block, topk, mode, scale, tau=0.0):
     B, Hq, N, d = Q.shape
-    return make_params(B, Hq, K.shape[1], N, d, block, topk, mode, Q.dtype, scale)
+    return make_params(B, Hq, K.shape[1], N, d, block, topk, mode, Q.dtype, scale, tau)
 
 
-def select(S, block=64, topk=0, mode="sparse", N=None, stream=None):
+def select(S, block=64, topk=0, mode="sparse", N=None, tau=0.0, stream=None):
     """K1: (idx, cnt, logg, slse) for S [B, Hq, Nb, Nb]."""
     lib = load_library()
     B, Hq, Nb, _ = S.shape
     N = N if N is not None else Nb * block
-    p = make_params(B, Hq, Hq, N, 64, block, topk, mode, torch.float32)
+    p = make_params(B, Hq, Hq, N, 64, block, topk, mode, torch.float32, tau=tau)
     dev = S.device
     idx = cnt = logg = None
-    if mode == "sparse":
+    if mode != "train":
         idx = torch.empty(B, Hq, Nb, topk, dtype=torch.int32, device=dev)
         cnt = torch.empty(B, Hq, Nb, dtype=torch.int32, device=dev)
         logg = torch.empty(B, Hq, Nb, topk, dtype=torch.float32, device=dev)
@@ -130,10 +132,10 @@ def select(S, block=64, topk=0, mode="sparse", N=None, stream=None):
 
 
 def forward(Q, K, V, S, block=64, mode="train", topk=0, scale=0.0, out=None, lse=None, ws=None,
-            stream=None):
+            tau=0.0, stream=None):
     """Gated attention forward: returns (O, LSE)."""
     lib = load_library()
-    p = _prefill_params(Q, K, S, block, topk, mode, scale)
+    p = _prefill_params(Q, K, S, block, topk, mode, scale, tau)
     O = out if out is not None else torch.empty_like(Q)
     LSE = lse if lse is not None else torch.empty(Q.shape[:3], dtype=torch.float32, device=Q.device)
     if ws is None:
@@ -159,12 +161,17 @@ def backward(Q, K, V, S, O, LSE, dO, block=64, scale=0.0, grads=None, ws=None, s
 
 
 def decode(q, Kc, Vc, S, L=None, block=64, topk=32, scale=0.0, num_splits=0, out=None, lse=None,
-           ws=None, stream=None):
-    """Sparse one-token decode: returns (O [B,Hq,d], LSE [B,Hq])."""
+           ws=None, tau=None, stream=None):
+    """Sparse one-token decode: returns (O [B,Hq,d], LSE [B,Hq]).
+
+    ``tau`` set selects threshold mode (blocks whose gate reaches tau, at most topk).
+    """
     lib = load_library()
     B, Hq, d = q.shape
     L = Kc.shape[2] if L is None else L
-    p = make_params(B, Hq, Kc.shape[1], L, d, block, topk, "sparse", q.dtype, scale)
+    mode = "sparse" if tau is None else "threshold"
+    p = make_params(B, Hq, Kc.shape[1], L, d, block, topk, mode, q.dtype, scale,
+                    0.0 if tau is None else tau)
     O = out if out is not None else torch.empty_like(q)
     LSE = lse if lse is not None else torch.empty(B, Hq, dtype=torch.float32, device=q.device)
     if ws is None:
@@ -196,7 +203,7 @@ def check(ws, stream=None):
 
 
 def decode_noalloc(q, Kc, Vc, S, L=None, block=64, topk=32, scale=0.0, num_splits=0, out=None,
-                   lse=None, stream=None):
+                   lse=None, tau=None, stream=None):
     """gbs_decode_noalloc: the decode with the library's own static scratch.
 
     For callers that cannot allocate device memory while decoding; see
@@ -209,7 +216,9 @@ def decode_noalloc(q, Kc, Vc, S, L=None, block=64, topk=32, scale=0.0, num_split
     f.argtypes = [ctypes.POINTER(Params), vp, vp, vp, vp, vp, vp, ctypes.c_int, vp]
     B, Hq, d = q.shape
     L = Kc.shape[2] if L is None else L
-    p = make_params(B, Hq, Kc.shape[1], L, d, block, topk, "sparse", q.dtype, scale)
+    mode = "sparse" if tau is None else "threshold"
+    p = make_params(B, Hq, Kc.shape[1], L, d, block, topk, mode, q.dtype, scale,
+                    0.0 if tau is None else tau)
     O = out if out is not None else torch.empty_like(q)
     LSE = lse if lse is not None else torch.empty(B, Hq, dtype=torch.float32, device=q.device)
     _check(f(ctypes.byref(p), _ptr(q), _ptr(Kc), _ptr(Vc), _ptr(S), _ptr(O), _ptr(LSE), num_splits,

@@ -85,6 +85,9 @@ extern "C" gbs_status gbs_decode_noalloc(const gbs_params* in, const void* q, co
   if (p.dtype != GBS_BF16 && p.dtype != GBS_F32) return noalloc_fail(GBS_ERR_INVALID_ARG, "unknown dtype");
   if (p.topk < 0 || p.topk > GBS_MAX_TOPK) return noalloc_fail(GBS_ERR_INVALID_ARG, "topk out of range");
   if (!(p.scale >= 0.f) || isinf(p.scale)) return noalloc_fail(GBS_ERR_INVALID_ARG, "bad scale");
+  const bool threshold = p.mode == GBS_THRESHOLD;
+  if (threshold && !(p.tau > 0.f && p.tau <= 1.f))
+    return noalloc_fail(GBS_ERR_INVALID_ARG, "threshold mode needs 0 < tau <= 1");
   if (num_splits < 0 || num_splits > kMaxSplitsNoalloc)
     return noalloc_fail(GBS_ERR_INVALID_ARG, "num_splits must be in [0, 8]");
   const void* ptrs[] = {q, Kc, Vc, S, O, LSE};
@@ -95,7 +98,8 @@ extern "C" gbs_status gbs_decode_noalloc(const gbs_params* in, const void* q, co
   gbs::Problem pr;
   pr.B = p.B; pr.Hq = p.Hq; pr.Hkv = p.Hkv; pr.N = p.N; pr.d = p.d; pr.bs = p.block;
   pr.Nb = (p.N + p.block - 1) / p.block; pr.G = p.Hq / p.Hkv; pr.topk = p.topk;
-  pr.mode = GBS_SPARSE; pr.dtype = p.dtype;
+  pr.mode = threshold ? GBS_THRESHOLD : GBS_SPARSE; pr.dtype = p.dtype;
+  pr.log_tau = threshold ? logf(p.tau) : 0.f;
   pr.scale = p.scale > 0.f ? p.scale : 1.0f / sqrtf((float)p.d);
   pr.scale_log2 = pr.scale * GBS_LOG2E;
 
@@ -134,8 +138,8 @@ extern "C" gbs_status gbs_decode_noalloc(const gbs_params* in, const void* q, co
   float* part_acc = reinterpret_cast<float*>(c);
 
   cudaStream_t st = (cudaStream_t)stream;
-  cudaError_t e = gbs::launch_select(S, (int)rows, pr.Nb, 1, cur, p.topk, true, sel.idx, sel.cnt,
-                                     sel.logg, nullptr, st);
+  cudaError_t e = gbs::launch_select(S, (int)rows, pr.Nb, 1, cur, p.topk, pr.mode, pr.log_tau,
+                                     sel.idx, sel.cnt, sel.logg, nullptr, st);
   if (e == cudaSuccess)
     e = gbs::launch_decode(pr, q, Kc, Vc, sel, cur, splits, part_ml, part_acc, O, LSE, st);
   if (e != cudaSuccess) return noalloc_fail(GBS_ERR_CUDA, cudaGetErrorString(e));

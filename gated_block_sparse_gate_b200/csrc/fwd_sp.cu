@@ -411,7 +411,7 @@ cudaError_t launch_sp(const SpArgs& a, const void* Q, const void* K, const void*
 }  // namespace
 
 bool fwd_sp_supported(const Problem& p) {
-  return p.dtype == GBS_BF16 && p.mode == GBS_SPARSE && p.bs == kSlot &&
+  return p.dtype == GBS_BF16 && p.mode != GBS_TRAIN && p.bs == kSlot &&
          (p.d == 64 || p.d == 128) && p.N % kSlot == 0 && p.G % 2 == 0;
 }
 

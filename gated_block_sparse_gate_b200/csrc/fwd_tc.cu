@@ -509,7 +509,7 @@ cudaError_t launch_fwd_tc(const Problem& p, const void* Q, const void* K, const 
   a.O = reinterpret_cast<__nv_bfloat16*>(O);
   a.LSE = LSE;
   a.err = err;
-  if (p.mode == GBS_SPARSE) {
+  if (p.mode != GBS_TRAIN) {
     const int n = p.B * p.Hq * a.n_tiles;
     plan_kernel<<<(n + 127) / 128, 128, 0, st>>>(p, sel, const_cast<int32_t*>(plan), plan_stride,
                                                  a.n_tiles);

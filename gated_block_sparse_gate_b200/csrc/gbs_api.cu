@@ -71,7 +71,7 @@ FwdWs carve_fwd(const Problem& p, void* ws) {
   FwdWs w{};
   const size_t rows = (size_t)p.B * p.Hq * p.Nb;
   w.sel.slse = c.take<float>(rows);
-  if (p.mode == GBS_SPARSE) {
+  if (p.mode != GBS_TRAIN) {
     w.sel.idx = c.take<int32_t>(rows * p.topk);
     w.sel.cnt = c.take<int32_t>(rows);
     w.sel.logg = c.take<float>(rows * p.topk);
@@ -115,12 +115,15 @@ gbs_status resolve(const gbs_params* in, int op, Problem* out) {
   if (q.B <= 0 || q.Hq <= 0 || q.Hkv <= 0 || q.N <= 0 || q.d <= 0 || q.block <= 0)
     return fail(GBS_ERR_INVALID_ARG, "B, Hq, Hkv, N, d and block must be positive");
   if (q.Hq % q.Hkv) return fail(GBS_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", q.Hq, q.Hkv);
-  if (q.mode != GBS_TRAIN && q.mode != GBS_SPARSE) return fail(GBS_ERR_INVALID_ARG, "mode %d unknown", q.mode);
+  if (q.mode != GBS_TRAIN && q.mode != GBS_SPARSE && q.mode != GBS_THRESHOLD)
+    return fail(GBS_ERR_INVALID_ARG, "mode %d unknown", q.mode);
+  if (q.mode == GBS_THRESHOLD && !(q.tau > 0.f && q.tau <= 1.f))
+    return fail(GBS_ERR_INVALID_ARG, "threshold mode needs 0 < tau <= 1 (got %g)", (double)q.tau);
   if (q.dtype != GBS_BF16 && q.dtype != GBS_F32) return fail(GBS_ERR_INVALID_ARG, "dtype %d unknown", q.dtype);
   if (!(q.scale >= 0.f) || isinf(q.scale)) return fail(GBS_ERR_INVALID_ARG, "scale must be finite and >= 0");
   if (op != GBS_OP_FWD && op != GBS_OP_BWD && op != GBS_OP_DECODE)
     return fail(GBS_ERR_INVALID_ARG, "op %d unknown", op);
-  const bool uses_topk = (op == GBS_OP_DECODE) || (q.mode == GBS_SPARSE);
+  const bool uses_topk = (op == GBS_OP_DECODE) || (q.mode != GBS_TRAIN);
   if (uses_topk && (q.topk < 0 || q.topk > GBS_MAX_TOPK))
     return fail(GBS_ERR_INVALID_ARG, "topk %d outside [0, %d]", q.topk, GBS_MAX_TOPK);
   if (op != GBS_OP_DECODE && q.N % q.block)
@@ -135,7 +138,10 @@ gbs_status resolve(const gbs_params* in, int op, Problem* out) {
   Problem& p = *out;
   p.B = q.B; p.Hq = q.Hq; p.Hkv = q.Hkv; p.N = q.N; p.d = q.d; p.bs = q.block;
   p.Nb = (int)Nb; p.G = q.Hq / q.Hkv; p.topk = uses_topk ? q.topk : 0;
-  p.mode = (op == GBS_OP_DECODE) ? GBS_SPARSE : q.mode; p.dtype = q.dtype;
+  p.mode = q.mode;
+  if (op == GBS_OP_DECODE && q.mode != GBS_THRESHOLD) p.mode = GBS_SPARSE;
+  p.dtype = q.dtype;
+  p.log_tau = p.mode == GBS_THRESHOLD ? logf(q.tau) : 0.f;
   p.scale = q.scale > 0.f ? q.scale : 1.0f / sqrtf((float)q.d);
   p.scale_log2 = p.scale * GBS_LOG2E;
   return GBS_OK;
@@ -231,14 +237,14 @@ gbs_status gbs_select(const gbs_params* in, const float* S, int32_t* idx, int32_
   Problem p;
   gbs_status s = resolve(in, GBS_OP_FWD, &p);
   if (s != GBS_OK) return s;
-  const bool sparse = p.mode == GBS_SPARSE;
+  const bool sparse = p.mode != GBS_TRAIN;
   if (!S) return fail(GBS_ERR_INVALID_ARG, "S is NULL");
   if (sparse && p.topk > 0 && (!idx || !logg)) return fail(GBS_ERR_INVALID_ARG, "idx/logg are NULL");
   if (sparse && !cnt) return fail(GBS_ERR_INVALID_ARG, "cnt is NULL");
   if (!sparse && !slse) return fail(GBS_ERR_INVALID_ARG, "slse is NULL in training mode");
   const int rows = p.B * p.Hq * p.Nb;
-  return cuda_status(launch_select(S, rows, p.Nb, p.Nb, -1, p.topk, sparse, idx, cnt, logg, slse,
-                                   (cudaStream_t)stream),
+  return cuda_status(launch_select(S, rows, p.Nb, p.Nb, -1, p.topk, p.mode, p.log_tau, idx, cnt,
+                                   logg, slse, (cudaStream_t)stream),
                      "gbs_select");
 }
 
@@ -255,10 +261,10 @@ gbs_status gbs_fwd(const gbs_params* in, const void* Q, const void* K, const voi
   if ((s = check_ws(ws, ws_bytes, w.bytes)) != GBS_OK) return s;
   w = carve_fwd(p, ws);
   cudaStream_t st = (cudaStream_t)stream;
-  const bool sparse = p.mode == GBS_SPARSE;
+  const bool sparse = p.mode != GBS_TRAIN;
   const int rows = p.B * p.Hq * p.Nb;
-  cudaError_t e = launch_select(S, rows, p.Nb, p.Nb, -1, p.topk, sparse, w.sel.idx, w.sel.cnt,
-                                w.sel.logg, sparse ? nullptr : w.sel.slse, st);
+  cudaError_t e = launch_select(S, rows, p.Nb, p.Nb, -1, p.topk, p.mode, p.log_tau, w.sel.idx,
+                                w.sel.cnt, w.sel.logg, sparse ? nullptr : w.sel.slse, st);
   if (e != cudaSuccess) return cuda_status(e, "gbs_fwd/select");
   if (fwd_tc2_supported(p)) {
     e = launch_fwd_tc2(p, Q, K, V, S, w.sel.slse, O, LSE, err_word(ws), st);
@@ -293,8 +299,8 @@ gbs_status gbs_bwd(const gbs_params* in, const void* Q, const void* K, const voi
   w = carve_bwd(p, ws);
   cudaStream_t st = (cudaStream_t)stream;
   const int rows = p.B * p.Hq * p.Nb;
-  cudaError_t e = launch_select(S, rows, p.Nb, p.Nb, -1, 0, false, nullptr, nullptr, nullptr,
-                                w.slse, st);
+  cudaError_t e = launch_select(S, rows, p.Nb, p.Nb, -1, 0, GBS_TRAIN, 0.f, nullptr, nullptr,
+                                nullptr, w.slse, st);
   if (e != cudaSuccess) return cuda_status(e, "gbs_bwd/select");
   if (bwd_tc_supported(p)) {
     e = launch_bwd_tc(p, Q, K, V, S, w.slse, O, LSE, dO, dQ, dK, dV, w.Dvec, w.Gblk, w.dQacc,
@@ -325,8 +331,8 @@ gbs_status gbs_decode(const gbs_params* in, const void* q, const void* Kc, const
   cudaStream_t st = (cudaStream_t)stream;
   const int BH = p.B * p.Hq;
   const int cur = (p.N - 1) / p.bs;
-  cudaError_t e = launch_select(S, BH, p.Nb, 1, cur, p.topk, true, w.sel.idx, w.sel.cnt,
-                                w.sel.logg, nullptr, st);
+  cudaError_t e = launch_select(S, BH, p.Nb, 1, cur, p.topk, p.mode, p.log_tau, w.sel.idx,
+                                w.sel.cnt, w.sel.logg, nullptr, st);
   if (e != cudaSuccess) return cuda_status(e, "gbs_decode/select");
   const int n_ent = (p.topk < cur ? p.topk : cur) + 1;
   int splits = num_splits;

@@ -22,6 +22,7 @@ struct Problem {
   int B, Hq, Hkv, N, d, bs, Nb, G, topk, mode, dtype;
   float scale;        // logit scale (natural units)
   float scale_log2;   // scale * log2(e)
+  float log_tau;      // threshold mode: ln(tau); 0 otherwise
 };
 
 // Selection buffers produced by K1 and read by the attention kernels.
@@ -32,12 +33,13 @@ struct Selection {
   float* logg;     // [B, Hq, Nb, topk]
 };
 
-// K1: gate normalisation (+ Top-K in sparse mode). rows_per_head = Nb for
-// prefill/training (row r has history r); for decode rows_per_head = 1 and
-// every row has history `decode_cur`.
+// K1: gate normalisation (+ Top-K in sparse and threshold modes; `mode` is a
+// gbs_mode, `log_tau` = ln(tau) is read in threshold mode only).
+// rows_per_head = Nb for prefill/training (row r has history r); for decode
+// rows_per_head = 1 and every row has history `decode_cur`.
 cudaError_t launch_select(const float* S, int n_rows, int row_stride, int rows_per_head,
-                          int decode_cur, int topk, bool sparse, int32_t* idx, int32_t* cnt,
-                          float* logg, float* slse, cudaStream_t st);
+                          int decode_cur, int topk, int mode, float log_tau, int32_t* idx,
+                          int32_t* cnt, float* logg, float* slse, cudaStream_t st);
 
 // Exact SIMT path (fp32 math for fp32 or bf16 storage).
 cudaError_t launch_fwd_simt(const Problem& p, const void* Q, const void* K, const void* V,

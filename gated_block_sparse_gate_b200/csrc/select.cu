@@ -16,6 +16,12 @@
 // log gates over the kept set. Comparisons are exact on the fp32 scores, so
 // the index lists are bit-identical to any other exact implementation of the
 // same ordering.
+//
+// Threshold mode (ai.viyan.live blog, section "Implementation and Efficiency":
+// only blocks whose importance passes a threshold are computed) first counts
+// the blocks whose training-mode log gate S[r,c] - lse_r reaches ln(tau); the
+// blocks passing are the highest-scoring ones, so the row then runs the same
+// Top-k with k = min(topk, that count).
 #include "common.cuh"
 #include "internal.h"
 
@@ -70,7 +76,7 @@ __device__ __forceinline__ int find_bin(const uint32_t* hist, int kk, int lane, 
 
 __global__ void __launch_bounds__(kWarps * 32)
 select_kernel(const float* __restrict__ S, int n_rows, int row_stride, int rows_per_head,
-              int decode_cur, int topk, int sparse, int32_t* __restrict__ idx,
+              int decode_cur, int topk, int mode, float log_tau, int32_t* __restrict__ idx,
               int32_t* __restrict__ cnt, float* __restrict__ logg, float* __restrict__ slse) {
   __shared__ uint32_t cache_all[kWarps][kRowCache];
   __shared__ uint32_t hist_all[kWarps][256];
@@ -86,18 +92,26 @@ select_kernel(const float* __restrict__ S, int n_rows, int row_stride, int rows_
   __syncwarp();
 
   // Training-mode normaliser over all of H_r.
-  if (slse) {
+  const bool threshold = mode == GBS_THRESHOLD;
+  float row_lse = -INFINITY;
+  if (slse || threshold) {
     float m = -INFINITY;
     for (int c = lane; c < r; c += 32) m = fmaxf(m, row_score(srow, cache, cached, c));
     m = warp_max(m);
     float s = 0.f;
     for (int c = lane; c < r; c += 32) s += expf(row_score(srow, cache, cached, c) - m);
     s = warp_sum(s);
-    if (lane == 0) slse[row] = r > 0 ? m + logf(s) : -INFINITY;
+    row_lse = r > 0 ? m + logf(s) : -INFINITY;
+    if (slse && lane == 0) slse[row] = row_lse;
   }
-  if (!sparse) return;
+  if (mode == GBS_TRAIN) return;
 
-  const int k = min(topk, r);
+  int k = min(topk, r);
+  if (threshold && k > 0) {
+    int n = 0;
+    for (int c = lane; c < r; c += 32) n += (row_score(srow, cache, cached, c) - row_lse) >= log_tau;
+    k = min(k, __reduce_add_sync(0xffffffffu, n));
+  }
   int32_t* out_idx = idx + (size_t)row * topk;
   float* out_logg = logg + (size_t)row * topk;
 
@@ -194,12 +208,12 @@ select_kernel(const float* __restrict__ S, int n_rows, int row_stride, int rows_
 }  // namespace
 
 cudaError_t launch_select(const float* S, int n_rows, int row_stride, int rows_per_head,
-                          int decode_cur, int topk, bool sparse, int32_t* idx, int32_t* cnt,
-                          float* logg, float* slse, cudaStream_t st) {
+                          int decode_cur, int topk, int mode, float log_tau, int32_t* idx,
+                          int32_t* cnt, float* logg, float* slse, cudaStream_t st) {
   if (n_rows <= 0) return cudaSuccess;
   const int grid = (n_rows + kWarps - 1) / kWarps;
   select_kernel<<<grid, kWarps * 32, 0, st>>>(S, n_rows, row_stride, rows_per_head, decode_cur,
-                                              topk, sparse ? 1 : 0, idx, cnt, logg, slse);
+                                              topk, mode, log_tau, idx, cnt, logg, slse);
   note_launch();
   return cudaGetLastError();
 }

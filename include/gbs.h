@@ -17,6 +17,14 @@
  *   - sparse mode attends only the Top-K historical blocks by score plus the
  *     current block (poster Abstract: fixed attention budget; HF page Abstract:
  *     hard Top-K). Gates are renormalised over the selected blocks.
+ *   - threshold mode is the dynamic variant (blog section "Implementation and
+ *     Efficiency": only blocks whose importance passes a threshold are
+ *     computed): a query block keeps the historical blocks whose training-mode
+ *     gate exp(S[r,c]) / sum_{c'<r} exp(S[r,c']) is at least tau, at most
+ *     topk of them (largest scores first), i.e. Top-k with
+ *     k = min(topk, #{c < r : gate >= tau}); gates are then renormalised over
+ *     the kept blocks as in sparse mode. The comparison is taken in fp32 as
+ *     S[r,c] - lse_r >= ln(tau), lse_r the fp32 row log-sum-exp.
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers (cudaMalloc / torch memory),
@@ -68,7 +76,7 @@ typedef enum gbs_status {
   GBS_ERR_WORKSPACE = 5      /* workspace missing or smaller than required      */
 } gbs_status;
 
-typedef enum gbs_mode { GBS_TRAIN = 0, GBS_SPARSE = 1 } gbs_mode;
+typedef enum gbs_mode { GBS_TRAIN = 0, GBS_SPARSE = 1, GBS_THRESHOLD = 2 } gbs_mode;
 typedef enum gbs_dtype { GBS_BF16 = 0, GBS_F32 = 1 } gbs_dtype;
 typedef enum gbs_op { GBS_OP_FWD = 0, GBS_OP_BWD = 1, GBS_OP_DECODE = 2 } gbs_op;
 
@@ -79,10 +87,11 @@ typedef struct gbs_params {
   int N;        /* tokens (training / prefill) or cache length L (decode)   */
   int d;        /* head dimension                                            */
   int block;    /* context-unit block size (tokens per block)               */
-  int topk;     /* sparse budget K of historical blocks (sparse / decode)   */
+  int topk;     /* budget K of historical blocks (sparse, threshold, decode) */
   int mode;     /* gbs_mode                                                  */
   int dtype;    /* gbs_dtype of Q, K, V, O, dO, dQ, dK, dV                   */
   float scale;  /* logit scale; 0 selects 1/sqrt(d)                          */
+  float tau;    /* threshold mode: gate threshold, 0 < tau <= 1; else unused */
 } gbs_params;
 
 /* Version as (major << 16) | minor. */
@@ -107,13 +116,14 @@ GBS_API gbs_status gbs_clear_error(void* ws, void* stream);
  * or the recorded status (GBS_ERR_TIMEOUT when a bounded wait expired). */
 GBS_API gbs_status gbs_check(const void* ws, void* stream);
 
-/* Gate normalisation and Top-K block selection (K1).
+/* Gate normalisation and Top-K (or threshold) block selection (K1).
  * Normalised softmax gates in log form over the attended historical set
  * (HF page Abstract; blog section "Differentiable Budget Constraints").
  *   S     [B, Hq, Nb, Nb] fp32, row r scores key blocks c < r.
  *   slse  [B, Hq, Nb] fp32 out: ln sum_{c<r} exp S[r, c] (-inf for r = 0);
- *         may be NULL in sparse mode.
- *   Sparse mode only (may be NULL in training mode):
+ *         may be NULL in sparse and threshold modes.
+ *   Sparse and threshold modes only (may be NULL in training mode); in
+ *   threshold mode read min(topk, r) below as k of the mode's definition:
  *   idx   [B, Hq, Nb, topk] int32 out: A_r ascending, -1 padded. A_r holds the
  *         min(topk, r) blocks c < r with the largest S[r, c]; ties go to the
  *         lower index; -0.0 equals +0.0.
@@ -127,8 +137,9 @@ GBS_API gbs_status gbs_select(const gbs_params* p, const float* S, int32_t* idx,
  *   Q [B,Hq,N,d], K/V [B,Hkv,N,d] in p->dtype; S [B,Hq,Nb,Nb] fp32.
  *   O [B,Hq,N,d] out (p->dtype); LSE [B,Hq,N] fp32 out, natural log of
  *   sum_j exp z_ij with z including scale and bias.
- *   p->mode selects training (every block c < r, gates over all of them) or
- *   sparse (Top-K blocks, gates renormalised over them).
+ *   p->mode selects training (every block c < r, gates over all of them),
+ *   sparse (Top-K blocks, gates renormalised over them) or threshold (blocks
+ *   whose gate reaches p->tau, at most Top-K, gates renormalised).
  *   ws: gbs_workspace_bytes(p, GBS_OP_FWD) bytes. */
 GBS_API gbs_status gbs_fwd(const gbs_params* p, const void* Q, const void* K, const void* V,
                    const float* S, void* O, float* LSE, void* ws, size_t ws_bytes,
@@ -150,6 +161,8 @@ GBS_API gbs_status gbs_bwd(const gbs_params* p, const void* Q, const void* K, co
  *   Nb = ceil(L / block): scores of the current block's row over key blocks
  *   c < cur = (L-1)/block. Attends the Top-K (p->topk) historical blocks with
  *   renormalised log gates plus the current block up to L-1 with bias 0.
+ *   p->mode GBS_THRESHOLD keeps only those of them whose gate reaches p->tau
+ *   (as in gbs_fwd); any other mode value selects plain Top-K.
  *   O [B,Hq,d] out (p->dtype); LSE [B,Hq] fp32 out.
  *   num_splits: partitions of the selected blocks per (b, h); 0 = automatic.
  *   ws: gbs_workspace_bytes(p, GBS_OP_DECODE) bytes. */

@@ -74,6 +74,26 @@ def test_invalid_params_rejected_before_launch(lib, kw, status):
     assert st == status, lib.gbs_last_error()
 
 
+@pytest.mark.parametrize("tau", [0.0, -0.5, 1.5, float("nan")])
+def test_threshold_mode_needs_tau_in_unit_interval(lib, tau):
+    p = gb.make_params(1, 4, 2, 256, 64, 64, 4, "threshold", tau=tau)
+    assert gb.workspace_bytes(p, gb.OP_FWD) == 0
+    assert gb.workspace_bytes(p, gb.OP_DECODE) == 0
+    fake = ctypes.c_void_p(4096)
+    st = lib.gbs_fwd(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, 1 << 30, None)
+    assert st == 1 and b"tau" in lib.gbs_last_error()
+
+
+def test_threshold_mode_workspace_matches_sparse(lib):
+    for op in (gb.OP_FWD, gb.OP_DECODE):
+        ps = gb.make_params(2, 8, 2, 4096, 128, 64, 16, "sparse")
+        pt = gb.make_params(2, 8, 2, 4096, 128, 64, 16, "threshold", tau=0.05)
+        assert gb.workspace_bytes(pt, op) == gb.workspace_bytes(ps, op) > 0
+    pt = gb.make_params(1, 4, 2, 256, 64, 64, 4, "threshold", tau=0.05)
+    ok = ctypes.c_void_p(4096)
+    assert lib.gbs_bwd(ctypes.byref(pt), *([ok] * 12), 1 << 30, None) == 2
+
+
 def test_null_and_misaligned_pointers_rejected(lib):
     p = gb.make_params(1, 4, 2, 256, 64, 64, 0, "train")
     ok = ctypes.c_void_p(4096)

@@ -98,14 +98,80 @@ def test_select_sparse_prefill_full_size_sampled(k):
             assert np.max(np.abs(logg[0, h, r, :len(A)] - lg), initial=0) < 1e-5
 
 
+# ------------------------------------------------------------ threshold select
+# The kernel decides S[r,c] - lse_r >= ln(tau) in fp32, the oracle in float64;
+# they can only disagree for a gate within rounding of tau. Rows with a gate
+# within THR_BAND (in log units) of ln(tau) are "boundary" rows: there the
+# kernel's count must lie between the two oracle counts of the band's edges and
+# its list must be the oracle's Top-k for that count; elsewhere bit-exact.
+# A row with one historical block has gate exactly 1 on both sides (its
+# log-sum-exp is the score itself), so it is never a boundary row.
+THR_BAND = 1e-4
+
+
+def _is_boundary(s, r, tau):
+    return r > 1 and (oracle.threshold_count(s, r, tau * math.exp(THR_BAND))
+                      != oracle.threshold_count(s, r, tau * math.exp(-THR_BAND)))
+
+
+def _threshold_rows_agree(Sn, idx, cnt, logg, k, tau, rows):
+    n_boundary = 0
+    for b, h, r in rows:
+        s = Sn[b, h, r]
+        lo = min(k, oracle.threshold_count(s, r, tau * math.exp(THR_BAND)))
+        hi = min(k, oracle.threshold_count(s, r, tau * math.exp(-THR_BAND)))
+        want = min(k, oracle.threshold_count(s, r, tau))
+        got = int(cnt[b, h, r])
+        if _is_boundary(s, r, tau) and lo != hi:
+            n_boundary += 1
+            assert lo <= got <= hi, (b, h, r, lo, got, hi)
+        else:
+            assert got == want, (b, h, r, got, want)
+        A = oracle.attended_blocks(s, r, oracle.SPARSE, got)
+        assert np.array_equal(idx[b, h, r, :got], A), (b, h, r)
+        assert np.all(idx[b, h, r, got:] == -1)
+        lg = oracle.log_gates(s, A, r)
+        assert np.max(np.abs(logg[b, h, r, :got] - lg), initial=0) < 1e-5
+    return n_boundary
+
+
+@pytest.mark.parametrize("tau", [1e-3, 0.02, 0.1, 0.5, 1.0])
+def test_select_threshold_tiny_workload(tau):
+    w = WORKLOADS["tiny_f32_n1024"]
+    S = make_prefill_inputs(w)["S"]
+    Sn = S.numpy()
+    rows = [(b, h, r) for b in range(S.shape[0]) for h in range(S.shape[1]) for r in range(16)]
+    for k in (0, 1, 3, 16):
+        idx, cnt, logg, _ = gb.select(S.to(DEV), topk=k, mode="threshold", tau=tau)
+        nb = _threshold_rows_agree(Sn, idx.cpu().numpy(), cnt.cpu().numpy(), logg.cpu().numpy(),
+                                   k, tau, rows)
+        assert nb == 0, nb  # this seed has no gate within the band of these taus
+
+
+@pytest.mark.parametrize("tau,k", [(0.01, 64), (0.002, 32), (0.05, 8)])
+def test_select_threshold_full_size_sampled(tau, k):
+    """Planted-score prefill workload (N=65536): sampled rows, threshold mode."""
+    w = WORKLOADS["sparse_prefill_bf16_n65536"]
+    S = make_prefill_inputs(w, with_grad=False)["S"]
+    idx, cnt, logg, _ = gb.select(S.to(DEV), topk=k, mode="threshold", tau=tau)
+    rng = np.random.default_rng(int(tau * 1e4) + k)
+    rows = [(0, h, int(r)) for h in (0, 13, 31)
+            for r in list(rng.integers(0, 1024, 40)) + [0, 1, 2, 50, 1023]]
+    nb = _threshold_rows_agree(S.numpy(), idx.cpu().numpy(), cnt.cpu().numpy(),
+                               logg.cpu().numpy(), k, tau, rows)
+    assert nb <= 2, nb
+    kept = cnt.cpu().numpy()[0, :, 64:]
+    assert kept.min() < min(k, 64) or tau <= 0.002  # the threshold does prune
+
+
 # ---------------------------------------------------------------------- forward
 
-def _check_fwd(x, mode, k, tol, rows=None):
+def _check_fwd(x, mode, k, tol, rows=None, tau=None):
     Qd, Kd, Vd, Sd = (x[n].to(DEV) for n in "QKVS")
-    O, LSE = gb.forward(Qd, Kd, Vd, Sd, mode=mode, topk=k)
+    O, LSE = gb.forward(Qd, Kd, Vd, Sd, mode=mode, topk=k, tau=0.0 if tau is None else tau)
     torch.cuda.synchronize()
     Or, Lr = oracle.gated_attention_forward(np64(x["Q"]), np64(x["K"]), np64(x["V"]), x["S"].numpy(),
-                                            64, mode=mode, topk=k, rows=rows)
+                                            64, mode=mode, topk=k, rows=rows, tau=tau)
     eo, el = rel_err(np64(O), Or), rel_err(LSE.cpu().numpy(), Lr)
     assert eo < tol and el < tol, (eo, el)
     return eo, el
@@ -157,6 +223,37 @@ def test_fwd_sparse_full_budget_matches_training():
     Qd, Kd, Vd, Sd = (x[n].to(DEV) for n in "QKVS")
     Ot, Lt = gb.forward(Qd, Kd, Vd, Sd, mode="train")
     Os, Ls = gb.forward(Qd, Kd, Vd, Sd, mode="sparse", topk=8)
+    torch.cuda.synchronize()
+    assert rel_err(np64(Os), np64(Ot)) < 1e-2 and rel_err(Ls.cpu().numpy(), Lt.cpu().numpy()) < 1e-5
+
+
+def _no_boundary_gates(S, tau):
+    """True when no gate of S lies within THR_BAND of tau (log units)."""
+    Sn = S.numpy()
+    B, H, Nb, _ = Sn.shape
+    return not any(_is_boundary(Sn[b, h, r], r, tau)
+                   for b in range(B) for h in range(H) for r in range(Nb))
+
+
+@pytest.mark.parametrize("shape,k,tau", [
+    ((1, 8, 2, 1024, 128), 6, 0.05),   # two tiles per CTA (G even)
+    ((2, 4, 4, 320, 64), 3, 0.2),      # G = 1: one tile per CTA
+    ((1, 4, 1, 448, 128), 100, 0.1),   # budget above every count: threshold alone
+    ((1, 4, 2, 512, 128), 4, 1.0),     # only a sole historical block passes
+])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_fwd_threshold(shape, k, tau, dtype):
+    B, Hq, Hkv, N, d = shape
+    x = _small(41 + k, B, Hq, Hkv, N, d, dtype, scaled=True)
+    assert _no_boundary_gates(x["S"], tau)
+    _check_fwd(x, "threshold", k, TOL_F32 if dtype == torch.float32 else TOL_BF16, tau=tau)
+
+
+def test_fwd_threshold_tiny_tau_equals_training():
+    x = _small(43, 1, 4, 2, 512, 128, torch.bfloat16, False)
+    Qd, Kd, Vd, Sd = (x[n].to(DEV) for n in "QKVS")
+    Ot, Lt = gb.forward(Qd, Kd, Vd, Sd, mode="train")
+    Os, Ls = gb.forward(Qd, Kd, Vd, Sd, mode="threshold", topk=8, tau=1e-30)
     torch.cuda.synchronize()
     assert rel_err(np64(Os), np64(Ot)) < 1e-2 and rel_err(Ls.cpu().numpy(), Lt.cpu().numpy()) < 1e-5
 
@@ -218,14 +315,15 @@ def test_bwd_train_full_size_one_group():
 
 # ----------------------------------------------------------------------- decode
 
-def _check_decode(x, L, k, tol, seqs, num_splits=0):
+def _check_decode(x, L, k, tol, seqs, num_splits=0, tau=None):
     O, LSE = gb.decode(x["q"].to(DEV), x["Kc"].to(DEV), x["Vc"].to(DEV), x["S"].to(DEV), L=L,
-                       topk=k, num_splits=num_splits)
+                       topk=k, num_splits=num_splits, tau=tau)
     torch.cuda.synchronize()
     Kc = x["Kc"][seqs].cpu() if x["Kc"].is_cuda else x["Kc"][seqs]
     Vc = x["Vc"][seqs].cpu() if x["Vc"].is_cuda else x["Vc"][seqs]
+    mode = oracle.SPARSE if tau is None else oracle.THRESHOLD
     Or, Lr = oracle.gated_decode(np64(x["q"][seqs]), np64(Kc), np64(Vc), x["S"][seqs].cpu().numpy(),
-                                 L, 64, k)
+                                 L, 64, k, mode=mode, tau=tau)
     eo = rel_err(np64(O[seqs]), Or)
     el = rel_err(LSE[seqs].cpu().numpy(), Lr)
     assert eo < tol and el < tol, (eo, el)
@@ -245,6 +343,18 @@ def test_decode_f32_small():
     w = replace(WORKLOADS["sparse_decode_bf16_b64_l131072"], B=2, N=2000, dtype="f32")
     x = make_decode_inputs(w, B=2, L=2000)
     _check_decode(x, 2000, 5, TOL_F32, seqs=[0, 1])
+
+
+@pytest.mark.parametrize("tau,k", [(0.01, 64), (0.05, 8), (1e-30, 256)])
+def test_decode_threshold_small(tau, k):
+    from dataclasses import replace
+    L = 8133
+    w = replace(WORKLOADS["sparse_decode_bf16_b64_l131072"], B=4, N=L)
+    x = make_decode_inputs(w, B=4, L=L)
+    cur = (L - 1) // 64
+    Sn = x["S"].numpy()
+    assert not any(_is_boundary(Sn[b, h], cur, tau) for b in range(4) for h in range(Sn.shape[1]))
+    _check_decode(x, L, k, TOL_BF16, seqs=[0, 1, 2, 3], tau=tau)
 
 
 def test_decode_full_size_sampled():
