@@ -145,10 +145,11 @@ def forward(Q, K, V, S, block=64, mode="train", topk=0, scale=0.0, out=None, lse
     return O, LSE
 
 
-def backward(Q, K, V, S, O, LSE, dO, block=64, scale=0.0, grads=None, ws=None, stream=None):
-    """Training-mode backward: returns (dQ, dK, dV, dS)."""
+def backward(Q, K, V, S, O, LSE, dO, block=64, scale=0.0, grads=None, ws=None, mode="train",
+             topk=0, tau=0.0, stream=None):
+    """Backward of ``forward`` with the same mode/topk/tau: returns (dQ, dK, dV, dS)."""
     lib = load_library()
-    p = _prefill_params(Q, K, S, block, 0, "train", scale)
+    p = _prefill_params(Q, K, S, block, topk, mode, scale, tau)
     if grads is None:
         grads = (torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V), torch.empty_like(S))
     dQ, dK, dV, dS = grads

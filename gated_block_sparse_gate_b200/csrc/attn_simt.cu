@@ -1,5 +1,5 @@
 // attn_simt.cu — exact fp32 SIMT path of the gated attention (forward and
-// training-mode backward).
+// backward).
 //
 // Logit of query i and key j: z_ij = scale * q_i.k_j + b_ij, where b_ij is the
 // normalised log gate of key block c(j) for query block r(i) when c(j) is an
@@ -8,7 +8,12 @@
 // Attention", "The Logit Injection Mechanism"; HF paper page of "SAS: Simple
 // Attention Sparsification via End-to-End Optimization of Context Ranking",
 // Abstract). Training mode attends every earlier block (NeurIPS 2026 poster
-// page, Abstract); sparse mode the Top-K list produced by K1.
+// page, Abstract); sparse mode the Top-K list produced by K1. The backward
+// reads the normaliser `nlse` (over H_r in training mode, over the kept blocks
+// A_r otherwise) and, outside training mode, the kept-block bitmap of K1: a
+// block outside A_r is skipped and its tile sum G is 0. The selection itself
+// is a discrete choice and passes no gradient; dS flows through the
+// renormalised gates of the kept blocks only.
 //
 // This path computes in fp32 on the CUDA cores with one thread per query (or
 // key) row and a 64-row block per CTA. It serves fp32 inputs, where tensor-core
@@ -23,6 +28,11 @@ namespace gbs {
 namespace {
 
 constexpr int kBS = 64;  // context-unit block size this path supports
+
+// Whether block c is kept for score row `row` (always, without a bitmap).
+__device__ __forceinline__ bool kept(const uint32_t* mbits, int mwords, size_t row, int c) {
+  return !mbits || ((__ldg(mbits + row * mwords + (c >> 5)) >> (c & 31)) & 1u);
+}
 
 template <typename T, int D>
 __device__ __forceinline__ void load_rows(float* dst, int ld, const T* src, int tid, int nthr) {
@@ -126,7 +136,7 @@ bwd_dq_kernel(Problem p, const T* __restrict__ Q, const T* __restrict__ K,
               const T* __restrict__ V, const float* __restrict__ S,
               const float* __restrict__ slse, const float* __restrict__ LSE,
               const T* __restrict__ dO, const float* __restrict__ Dvec, T* __restrict__ dQ,
-              float* __restrict__ Gblk) {
+              float* __restrict__ Gblk, const uint32_t* __restrict__ mbits, int mwords) {
   extern __shared__ float smem[];
   float* Qs = smem;                   // [64][D+1]
   float* dOs = Qs + kBS * (D + 1);    // [64][D+1]
@@ -150,6 +160,10 @@ bwd_dq_kernel(Problem p, const T* __restrict__ Q, const T* __restrict__ K,
 
   for (int c = 0; c <= r; ++c) {
     const bool diag = c == r;
+    if (!diag && !kept(mbits, mwords, row_id, c)) {  // uniform over the CTA
+      if (t == 0) Gblk[row_id * p.Nb + c] = 0.f;
+      continue;
+    }
     const float bias = diag ? 0.f : S[row_id * p.Nb + c] - slse[row_id];
     __syncthreads();
     load_rows<T, D>(Ks, D, K + kvbase + (size_t)c * kBS * D, t, kBS);
@@ -189,7 +203,7 @@ bwd_dkdv_kernel(Problem p, const T* __restrict__ Q, const T* __restrict__ K,
                 const T* __restrict__ V, const float* __restrict__ S,
                 const float* __restrict__ slse, const float* __restrict__ LSE,
                 const T* __restrict__ dO, const float* __restrict__ Dvec, T* __restrict__ dK,
-                T* __restrict__ dV) {
+                T* __restrict__ dV, const uint32_t* __restrict__ mbits, int mwords) {
   constexpr int H2 = D / 2;
   extern __shared__ float smem[];
   float* Ks = smem;                    // [64][D+1] own key block
@@ -213,6 +227,7 @@ bwd_dkdv_kernel(Problem p, const T* __restrict__ Q, const T* __restrict__ K,
     for (int r = c; r < p.Nb; ++r) {
       const size_t row_id = (size_t)(b * p.Hq + h) * p.Nb + r;
       const bool diag = r == c;
+      if (!diag && !kept(mbits, mwords, row_id, c)) continue;  // uniform over the CTA
       const float bias2 = (diag ? 0.f : S[row_id * p.Nb + c] - slse[row_id]) * GBS_LOG2E;
       __syncthreads();
       load_rows<T, D>(Qs, D, Q + qbase + (size_t)r * kBS * D, t, 2 * kBS);
@@ -248,10 +263,12 @@ bwd_dkdv_kernel(Problem p, const T* __restrict__ Q, const T* __restrict__ K,
   }
 }
 
-// dS[r, c'] = G[r, c'] - g[r, c'] * sum_{c<r} G[r, c], 0 for c' >= r.
+// dS[r, c'] = G[r, c'] - g[r, c'] * sum_{c<r} G[r, c] for kept c' < r, else 0
+// (G is 0 outside the kept set, so the sum runs over it).
 __global__ void ds_finalize_kernel(const float* __restrict__ S, const float* __restrict__ slse,
                                    const float* __restrict__ Gblk, float* __restrict__ dS,
-                                   int Nb, size_t rows) {
+                                   int Nb, size_t rows, const uint32_t* __restrict__ mbits,
+                                   int mwords) {
   const size_t row = (size_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -262,7 +279,8 @@ __global__ void ds_finalize_kernel(const float* __restrict__ S, const float* __r
   tot = warp_sum(tot);
   const float lse = slse[row];
   for (int c = lane; c < Nb; c += 32)
-    dS[row * Nb + c] = c < r ? g[c] - expf(S[row * Nb + c] - lse) * tot : 0.f;
+    dS[row * Nb + c] =
+        (c < r && kept(mbits, mwords, row, c)) ? g[c] - expf(S[row * Nb + c] - lse) * tot : 0.f;
 }
 
 template <typename T, int D>
@@ -283,7 +301,7 @@ template <typename T, int D>
 cudaError_t bwd_simt_typed(const Problem& p, const void* Q, const void* K, const void* V,
                            const float* S, const float* slse, const void* O, const float* LSE,
                            const void* dO, void* dQ, void* dK, void* dV, float* dS, float* Dvec,
-                           float* Gblk, cudaStream_t st) {
+                           float* Gblk, const uint32_t* mbits, int mwords, cudaStream_t st) {
   const size_t rows = (size_t)p.B * p.Hq * p.N;
   bwd_dot_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>((const T*)O, (const T*)dO,
                                                                    Dvec, rows);
@@ -297,7 +315,8 @@ cudaError_t bwd_simt_typed(const Problem& p, const void* Q, const void* K, const
     if (e != cudaSuccess) return e;
     timer_begin(GBS_OP_BWD, st);
     kern<<<dim3(p.Nb, p.Hq, p.B), kBS, smem, st>>>(p, (const T*)Q, (const T*)K, (const T*)V, S,
-                                                    slse, LSE, (const T*)dO, Dvec, (T*)dQ, Gblk);
+                                                    slse, LSE, (const T*)dO, Dvec, (T*)dQ, Gblk,
+                                                    mbits, mwords);
     note_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -308,13 +327,14 @@ cudaError_t bwd_simt_typed(const Problem& p, const void* Q, const void* K, const
     if (e != cudaSuccess) return e;
     kern<<<dim3(p.Nb, p.Hkv, p.B), 2 * kBS, smem, st>>>(p, (const T*)Q, (const T*)K, (const T*)V,
                                                          S, slse, LSE, (const T*)dO, Dvec,
-                                                         (T*)dK, (T*)dV);
+                                                         (T*)dK, (T*)dV, mbits, mwords);
     note_launch();
     timer_end(GBS_OP_BWD, st);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   const size_t srows = (size_t)p.B * p.Hq * p.Nb;
-  ds_finalize_kernel<<<(unsigned)((srows + 7) / 8), 256, 0, st>>>(S, slse, Gblk, dS, p.Nb, srows);
+  ds_finalize_kernel<<<(unsigned)((srows + 7) / 8), 256, 0, st>>>(S, slse, Gblk, dS, p.Nb, srows,
+                                                                  mbits, mwords);
   note_launch();
   return cudaGetLastError();
 }
@@ -322,9 +342,11 @@ cudaError_t bwd_simt_typed(const Problem& p, const void* Q, const void* K, const
 }  // namespace
 
 cudaError_t launch_ds_finalize(const Problem& p, const float* S, const float* slse,
-                               const float* Gblk, float* dS, cudaStream_t st) {
+                               const float* Gblk, float* dS, const uint32_t* mbits, int mwords,
+                               cudaStream_t st) {
   const size_t srows = (size_t)p.B * p.Hq * p.Nb;
-  ds_finalize_kernel<<<(unsigned)((srows + 7) / 8), 256, 0, st>>>(S, slse, Gblk, dS, p.Nb, srows);
+  ds_finalize_kernel<<<(unsigned)((srows + 7) / 8), 256, 0, st>>>(S, slse, Gblk, dS, p.Nb, srows,
+                                                                  mbits, mwords);
   note_launch();
   return cudaGetLastError();
 }
@@ -346,10 +368,12 @@ cudaError_t launch_fwd_simt(const Problem& p, const void* Q, const void* K, cons
 cudaError_t launch_bwd_simt(const Problem& p, const void* Q, const void* K, const void* V,
                             const float* S, const float* slse, const void* O, const float* LSE,
                             const void* dO, void* dQ, void* dK, void* dV, float* dS,
-                            float* Dvec, float* Gblk, cudaStream_t st) {
+                            float* Dvec, float* Gblk, const uint32_t* mbits, int mwords,
+                            cudaStream_t st) {
   if (p.bs != kBS) return cudaErrorNotSupported;
 #define GBS_BWD(T, DD)                                                                       \
-  return bwd_simt_typed<T, DD>(p, Q, K, V, S, slse, O, LSE, dO, dQ, dK, dV, dS, Dvec, Gblk, st)
+  return bwd_simt_typed<T, DD>(p, Q, K, V, S, slse, O, LSE, dO, dQ, dK, dV, dS, Dvec, Gblk,   \
+                               mbits, mwords, st)
   if (p.dtype == GBS_F32) {
     if (p.d == 64) GBS_BWD(float, 64);
     if (p.d == 128) GBS_BWD(float, 128);

@@ -35,6 +35,14 @@
 // 9 TMEM allocator + MMA issuer, 10-13 dQ drain (lane quadrant w%4): the
 // drain warps move dQ out of TMEM while the compute warps start the next
 // step. Every mbarrier wait is bounded.
+//
+// Sparse and threshold modes (the gradient through the gates renormalised
+// over the kept blocks A_r; the selection itself passes no gradient) run the
+// same kernel over a step list: bwd_plan_kernel lists, per key tile, the
+// (q-head, query tile) pairs in which some query block keeps one of the tile's
+// two key blocks (plus the diagonal tile), and a compute warp whose (query
+// block, key block) pair is not kept treats it as masked, so its P, dZ and G
+// are 0.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -98,8 +106,51 @@ struct BwdArgs {
   __nv_bfloat16* dK;
   __nv_bfloat16* dV;
   int n_tiles;  // 128-row tiles per head (keys and queries alike)
+  const uint32_t* mbits;  // kept-block bitmap (null in training mode)
+  int mwords;
+  const int32_t* plan;    // per-CTA step lists (null in training mode)
+  int plan_stride;
   unsigned int* err;
 };
+
+// Step list of CTA (key tile u, batch x kv-head bk): entry 0 is the count,
+// then (q-head in group << 16 | query tile) for every query tile t >= u of
+// every q-head where some query block of t keeps a key block of u; t = u (the
+// diagonal) always. One warp per CTA (id = u * BKV + bk, the attention
+// kernel's block index), ballot compaction in t order.
+__global__ void bwd_plan_kernel(const uint32_t* __restrict__ mbits, int mwords, int Nb, int n_tiles,
+                                int G, int Hq, int Hkv, int BKV, int32_t* __restrict__ plan,
+                                int plan_stride) {
+  const int lane = threadIdx.x & 31;
+  const int id = (int)(blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5));
+  if (id >= n_tiles * BKV) return;
+  const int u = id / BKV, bk = id % BKV;
+  const int b = bk / Hkv, kvh = bk % Hkv;
+  int32_t* out = plan + (size_t)id * plan_stride;
+  const int cw = (2 * u) >> 5, sh = (2 * u) & 31;
+  const uint32_t lanes_below = (1u << lane) - 1u;
+  int n = 0;
+  for (int hh = 0; hh < G; ++hh) {
+    const size_t rowbase = (size_t)(b * Hq + kvh * G + hh) * Nb;
+    for (int t0 = u; t0 < n_tiles; t0 += 32) {
+      const int t = t0 + lane;
+      bool need = false;
+      if (t < n_tiles) {
+        if (t == u) {
+          need = true;
+        } else {
+          need = (__ldg(mbits + (rowbase + 2 * t) * mwords + cw) >> sh) & 3u;
+          if (!need && 2 * t + 1 < Nb)
+            need = (__ldg(mbits + (rowbase + 2 * t + 1) * mwords + cw) >> sh) & 3u;
+        }
+      }
+      const uint32_t m = __ballot_sync(0xffffffffu, need);
+      if (need) out[1 + n + __popc(m & lanes_below)] = (hh << 16) | t;
+      n += __popc(m);
+    }
+  }
+  if (lane == 0) out[0] = n;
+}
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -134,7 +185,19 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const int bk = (int)(blockIdx.x % BKV);
   const int b = bk / p.Hkv, kvh = bk % p.Hkv;
   const int per_head = a.n_tiles - u;
-  const int n_steps = p.G * per_head;
+  const int32_t* steps = a.plan ? a.plan + (size_t)blockIdx.x * a.plan_stride : nullptr;
+  const int n_steps = steps ? __ldg(steps) : p.G * per_head;
+  // (q-head within the group, query tile) of step j
+  auto step_at = [&](int j, int& hh, int& t) {
+    if (steps) {
+      const int e = __ldg(steps + 1 + j);
+      hh = e >> 16;
+      t = e & 0xffff;
+    } else {
+      hh = j / per_head;
+      t = u + j % per_head;
+    }
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
@@ -183,8 +246,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const int sj = jj % kQStages;
         if (!mbar_wait(&bars->staged[sj], (jj / kQStages) & 1, abort_flag, a.err, kTimeoutNs))
           return false;
-        const int t = u + jj % per_head;
-        const int bh = b * p.Hq + kvh * p.G + jj / per_head;
+        int hh, t;
+        step_at(jj, hh, t);
+        const int bh = b * p.Hq + kvh * p.G + hh;
 #pragma unroll 1
         for (int w = 0; w < kComputeWarps; ++w) {
           const int quad = w & 3, hq = w >> 2;
@@ -210,7 +274,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           }
           bulk_wait_group_read0();
         }
-        const int hh = j / per_head, t = u + j % per_head;
+        int hh, t;
+        step_at(j, hh, t);
         const int bh = b * p.Hq + kvh * p.G + hh;
         const int q0 = t * kBQ;
         // rows past the end are never read: a half tile past N is fully masked
@@ -326,17 +391,20 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     bool ok = true;
     for (int j = 0; j < n_steps; ++j) {
       const int st = j % kQStages;
-      const int hh = j / per_head, t = u + j % per_head;
+      int hh, t;
+      step_at(j, hh, t);
       const int bh = b * p.Hq + kvh * p.G + hh;
       const int r = 2 * t + hq;  // this warp's query block
+      const size_t row = (size_t)bh * p.Nb + r;
       int mode = kFull;
       float bias2 = 0.f;
       if (r >= p.Nb || cj > r) {
         mode = kMasked;
       } else if (cj == r) {
         mode = kCausal;
+      } else if (a.mbits && !((__ldg(a.mbits + row * a.mwords + (cj >> 5)) >> (cj & 31)) & 1u)) {
+        mode = kMasked;  // key block not kept for this query block
       } else {
-        const size_t row = (size_t)bh * p.Nb + r;
         bias2 = (__ldg(a.S + row * p.Nb + cj) - __ldg(a.slse + row)) * GBS_LOG2E;
       }
       if (!mbar_wait(&bars->s_full, j & 1, abort_flag, a.err, kTimeoutNs) ||
@@ -627,14 +695,23 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, const void* Q, const void* K, con
 
 bool bwd_tc_supported(const Problem& p) {
   return p.dtype == GBS_BF16 && p.bs == 64 && (p.d == 64 || p.d == 128) && p.N % 64 == 0 &&
-         p.mode == GBS_TRAIN;
+         (p.Nb + 1) / 2 < 65536;
+}
+
+size_t bwd_plan_ints(const Problem& p) {
+  if (p.mode == GBS_TRAIN) return 0;
+  const size_t n_tiles = (size_t)(p.Nb + 1) / 2;
+  return (size_t)p.B * p.Hkv * n_tiles * (1 + (size_t)p.G * n_tiles);
 }
 
 cudaError_t launch_bwd_tc(const Problem& p, const void* Q, const void* K, const void* V,
                           const float* S, const float* slse, const void* O, const float* LSE,
                           const void* dO, void* dQ, void* dK, void* dV, float* Dvec, float* Gblk,
-                          float* dQacc, unsigned int* err, cudaStream_t st) {
+                          float* dQacc, const uint32_t* mbits, int mwords, int32_t* plan,
+                          unsigned int* err, cudaStream_t st) {
   if (!bwd_tc_supported(p)) return cudaErrorNotSupported;
+  const bool sparse = p.mode != GBS_TRAIN;
+  if (sparse && (!mbits || !plan)) return cudaErrorInvalidValue;
   BwdArgs a;
   a.p = p;
   a.S = S;
@@ -646,7 +723,19 @@ cudaError_t launch_bwd_tc(const Problem& p, const void* Q, const void* K, const 
   a.dK = reinterpret_cast<__nv_bfloat16*>(dK);
   a.dV = reinterpret_cast<__nv_bfloat16*>(dV);
   a.n_tiles = (p.Nb + 1) / 2;
+  a.mbits = sparse ? mbits : nullptr;
+  a.mwords = mwords;
+  a.plan = sparse ? plan : nullptr;
+  a.plan_stride = 1 + p.G * a.n_tiles;
   a.err = err;
+  if (sparse) {
+    const int ctas = p.B * p.Hkv * a.n_tiles;
+    bwd_plan_kernel<<<(unsigned)((ctas + 7) / 8), 256, 0, st>>>(
+        mbits, mwords, p.Nb, a.n_tiles, p.G, p.Hq, p.Hkv, p.B * p.Hkv, plan, a.plan_stride);
+    note_launch();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   cudaError_t e = cudaMemsetAsync(dQacc, 0, (size_t)p.B * p.Hq * p.N * p.d * sizeof(float), st);
   if (e == cudaSuccess)
     e = cudaMemsetAsync(Gblk, 0, (size_t)p.B * p.Hq * p.Nb * p.Nb * sizeof(float), st);

@@ -55,9 +55,14 @@ struct FwdWs {
   size_t bytes;
 };
 struct BwdWs {
-  float *slse, *Dvec, *Gblk, *dQacc;
+  float *slse, *Dvec, *Gblk, *dQacc;  // slse: gate normaliser (over H_r, or over A_r)
+  Selection sel;                      // outside training mode: K1's lists
+  uint32_t* mbits;                    // outside training mode: kept-block bitmap
+  int32_t* plan;                      // outside training mode, tensor-core path: step lists
   size_t bytes;
 };
+
+inline int mask_words(const Problem& p) { return (p.Nb + 31) / 32; }
 struct DecWs {
   Selection sel;
   float *part_ml, *part_acc;
@@ -89,6 +94,14 @@ BwdWs carve_bwd(const Problem& p, void* ws) {
   w.Dvec = c.take<float>((size_t)p.B * p.Hq * p.N);
   w.Gblk = c.take<float>((size_t)p.B * p.Hq * p.Nb * p.Nb);
   if (bwd_tc_supported(p)) w.dQacc = c.take<float>((size_t)p.B * p.Hq * p.N * p.d);
+  if (p.mode != GBS_TRAIN) {
+    const size_t rows = (size_t)p.B * p.Hq * p.Nb;
+    w.sel.idx = c.take<int32_t>(rows * p.topk);
+    w.sel.cnt = c.take<int32_t>(rows);
+    w.sel.logg = c.take<float>(rows * p.topk);
+    w.mbits = c.take<uint32_t>(rows * mask_words(p));
+    if (bwd_tc_supported(p)) w.plan = c.take<int32_t>(bwd_plan_ints(p));
+  }
   w.bytes = c.off;
   return w;
 }
@@ -130,8 +143,6 @@ gbs_status resolve(const gbs_params* in, int op, Problem* out) {
     return fail(GBS_ERR_INVALID_ARG, "N (%d) must be a multiple of block (%d)", q.N, q.block);
   if (q.block != 64) return fail(GBS_ERR_UNSUPPORTED, "block %d: only 64 is built", q.block);
   if (q.d != 64 && q.d != 128) return fail(GBS_ERR_UNSUPPORTED, "d %d: only 64 and 128 are built", q.d);
-  if (op == GBS_OP_BWD && q.mode != GBS_TRAIN)
-    return fail(GBS_ERR_UNSUPPORTED, "the backward pass is built for training mode only");
   const size_t Nb = ((size_t)q.N + q.block - 1) / q.block;
   if ((size_t)q.B * q.Hq * Nb * Nb > ((size_t)1 << 40) || (size_t)q.B * q.Hq * q.N * q.d > ((size_t)1 << 40))
     return fail(GBS_ERR_INVALID_ARG, "problem too large");
@@ -299,17 +310,23 @@ gbs_status gbs_bwd(const gbs_params* in, const void* Q, const void* K, const voi
   w = carve_bwd(p, ws);
   cudaStream_t st = (cudaStream_t)stream;
   const int rows = p.B * p.Hq * p.Nb;
-  cudaError_t e = launch_select(S, rows, p.Nb, p.Nb, -1, 0, GBS_TRAIN, 0.f, nullptr, nullptr,
-                                nullptr, w.slse, st);
+  const int mwords = mask_words(p);
+  cudaError_t e;
+  if (p.mode == GBS_TRAIN)
+    e = launch_select(S, rows, p.Nb, p.Nb, -1, 0, GBS_TRAIN, 0.f, nullptr, nullptr, nullptr,
+                      w.slse, st);
+  else  // the forward's selection, recomputed: normaliser over A_r and the kept bitmap
+    e = launch_select(S, rows, p.Nb, p.Nb, -1, p.topk, p.mode, p.log_tau, w.sel.idx, w.sel.cnt,
+                      w.sel.logg, nullptr, st, w.slse, w.mbits, mwords);
   if (e != cudaSuccess) return cuda_status(e, "gbs_bwd/select");
   if (bwd_tc_supported(p)) {
     e = launch_bwd_tc(p, Q, K, V, S, w.slse, O, LSE, dO, dQ, dK, dV, w.Dvec, w.Gblk, w.dQacc,
-                      err_word(ws), st);
-    if (e == cudaSuccess) e = launch_ds_finalize(p, S, w.slse, w.Gblk, dS, st);
+                      w.mbits, mwords, w.plan, err_word(ws), st);
+    if (e == cudaSuccess) e = launch_ds_finalize(p, S, w.slse, w.Gblk, dS, w.mbits, mwords, st);
     return cuda_status(e, "gbs_bwd");
   }
   return cuda_status(launch_bwd_simt(p, Q, K, V, S, w.slse, O, LSE, dO, dQ, dK, dV, dS, w.Dvec,
-                                     w.Gblk, st),
+                                     w.Gblk, w.mbits, mwords, st),
                      "gbs_bwd");
 }
 

@@ -36,10 +36,14 @@ struct Selection {
 // K1: gate normalisation (+ Top-K in sparse and threshold modes; `mode` is a
 // gbs_mode, `log_tau` = ln(tau) is read in threshold mode only).
 // rows_per_head = Nb for prefill/training (row r has history r); for decode
-// rows_per_head = 1 and every row has history `decode_cur`.
+// rows_per_head = 1 and every row has history `decode_cur`. Sparse and
+// threshold modes can also write sel_lse [rows] (the log-sum-exp of S over
+// the kept blocks) and mbits [rows, mwords] (bit c of word c/32 set when block
+// c is kept; every word written).
 cudaError_t launch_select(const float* S, int n_rows, int row_stride, int rows_per_head,
                           int decode_cur, int topk, int mode, float log_tau, int32_t* idx,
-                          int32_t* cnt, float* logg, float* slse, cudaStream_t st);
+                          int32_t* cnt, float* logg, float* slse, cudaStream_t st,
+                          float* sel_lse = nullptr, uint32_t* mbits = nullptr, int mwords = 0);
 
 // Exact SIMT path (fp32 math for fp32 or bf16 storage).
 cudaError_t launch_fwd_simt(const Problem& p, const void* Q, const void* K, const void* V,
@@ -48,7 +52,8 @@ cudaError_t launch_fwd_simt(const Problem& p, const void* Q, const void* K, cons
 cudaError_t launch_bwd_simt(const Problem& p, const void* Q, const void* K, const void* V,
                             const float* S, const float* slse, const void* O, const float* LSE,
                             const void* dO, void* dQ, void* dK, void* dV, float* dS,
-                            float* Dvec, float* Gblk, cudaStream_t st);
+                            float* Dvec, float* Gblk, const uint32_t* mbits, int mwords,
+                            cudaStream_t st);
 
 // Decode (split over the selected blocks, then combine).
 cudaError_t launch_decode(const Problem& p, const void* q, const void* Kc, const void* Vc,
@@ -77,13 +82,21 @@ cudaError_t launch_fwd_sp(const Problem& p, const void* Q, const void* K, const 
                           const Selection& sel, int32_t* plan, int plan_stride, void* O,
                           float* LSE, unsigned int* err, cudaStream_t st);
 bool fwd_sp_supported(const Problem& p);
+// Backward. `slse` is the gate normaliser (over H_r in training mode, over the
+// kept blocks otherwise); outside training mode `mbits` is K1's kept-block
+// bitmap and `plan` a workspace of bwd_plan_ints(p) ints where the launcher
+// lists, per (batch, kv-head, 128-key tile), the (q-head, 128-query tile)
+// steps that touch a kept block.
 cudaError_t launch_bwd_tc(const Problem& p, const void* Q, const void* K, const void* V,
                           const float* S, const float* slse, const void* O, const float* LSE,
                           const void* dO, void* dQ, void* dK, void* dV, float* Dvec, float* Gblk,
-                          float* dQacc, unsigned int* err, cudaStream_t st);
+                          float* dQacc, const uint32_t* mbits, int mwords, int32_t* plan,
+                          unsigned int* err, cudaStream_t st);
 bool bwd_tc_supported(const Problem& p);
-// dS from the tile sums G (shared by both backward paths).
+size_t bwd_plan_ints(const Problem& p);
+// dS from the tile sums G (shared by both backward paths); mbits as above.
 cudaError_t launch_ds_finalize(const Problem& p, const float* S, const float* slse,
-                               const float* Gblk, float* dS, cudaStream_t st);
+                               const float* Gblk, float* dS, const uint32_t* mbits, int mwords,
+                               cudaStream_t st);
 
 }  // namespace gbs

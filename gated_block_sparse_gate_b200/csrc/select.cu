@@ -22,6 +22,10 @@
 // the blocks whose training-mode log gate S[r,c] - lse_r reaches ln(tau); the
 // blocks passing are the highest-scoring ones, so the row then runs the same
 // Top-k with k = min(topk, that count).
+//
+// For the sparse backward the kernel can also emit, per row, the normaliser
+// over the kept set (sel_lse) and a bitmap of the kept blocks (bit c of word
+// c / 32, every word of the row written).
 #include "common.cuh"
 #include "internal.h"
 
@@ -77,7 +81,8 @@ __device__ __forceinline__ int find_bin(const uint32_t* hist, int kk, int lane, 
 __global__ void __launch_bounds__(kWarps * 32)
 select_kernel(const float* __restrict__ S, int n_rows, int row_stride, int rows_per_head,
               int decode_cur, int topk, int mode, float log_tau, int32_t* __restrict__ idx,
-              int32_t* __restrict__ cnt, float* __restrict__ logg, float* __restrict__ slse) {
+              int32_t* __restrict__ cnt, float* __restrict__ logg, float* __restrict__ slse,
+              float* __restrict__ sel_lse, uint32_t* __restrict__ mbits, int mwords) {
   __shared__ uint32_t cache_all[kWarps][kRowCache];
   __shared__ uint32_t hist_all[kWarps][256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -169,7 +174,8 @@ select_kernel(const float* __restrict__ S, int n_rows, int row_stride, int rows_
   int written = 0, eq_seen = 0;
   float m = -INFINITY;
   const uint32_t lanes_below = (1u << lane) - 1u;
-  for (int base = 0; base < r && written < k; base += 32) {
+  int base = 0;
+  for (; base < r && written < k; base += 32) {
     const int c = base + lane;
     const bool valid = c < r;
     const float s = valid ? row_score(srow, cache, cached, c) : 0.f;
@@ -180,6 +186,7 @@ select_kernel(const float* __restrict__ S, int n_rows, int row_stride, int rows_
     const bool keep = valid && (k >= r || u > T || (eq && eq_before < need_eq));
     eq_seen += __popc(eq_mask);
     const uint32_t keep_mask = __ballot_sync(0xffffffffu, keep);
+    if (mbits && lane == 0) mbits[(size_t)row * mwords + (base >> 5)] = keep_mask;
     const int pos = written + __popc(keep_mask & lanes_below);
     if (keep) {
       out_idx[pos] = c;
@@ -203,17 +210,22 @@ select_kernel(const float* __restrict__ S, int n_rows, int row_stride, int rows_
     }
   }
   if (lane == 0) cnt[row] = k;
+  if (sel_lse && lane == 0) sel_lse[row] = lse;
+  if (mbits)
+    for (int wi = (base >> 5) + lane; wi < mwords; wi += 32) mbits[(size_t)row * mwords + wi] = 0u;
 }
 
 }  // namespace
 
 cudaError_t launch_select(const float* S, int n_rows, int row_stride, int rows_per_head,
                           int decode_cur, int topk, int mode, float log_tau, int32_t* idx,
-                          int32_t* cnt, float* logg, float* slse, cudaStream_t st) {
+                          int32_t* cnt, float* logg, float* slse, cudaStream_t st,
+                          float* sel_lse, uint32_t* mbits, int mwords) {
   if (n_rows <= 0) return cudaSuccess;
   const int grid = (n_rows + kWarps - 1) / kWarps;
   select_kernel<<<grid, kWarps * 32, 0, st>>>(S, n_rows, row_stride, rows_per_head, decode_cur,
-                                              topk, mode, log_tau, idx, cnt, logg, slse);
+                                              topk, mode, log_tau, idx, cnt, logg, slse, sel_lse,
+                                              mbits, mwords);
   note_launch();
   return cudaGetLastError();
 }

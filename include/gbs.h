@@ -145,11 +145,17 @@ GBS_API gbs_status gbs_fwd(const gbs_params* p, const void* Q, const void* K, co
                    const float* S, void* O, float* LSE, void* ws, size_t ws_bytes,
                    void* stream);
 
-/* Gated attention backward, training mode (p->mode must be GBS_TRAIN).
- *   O, LSE: outputs of gbs_fwd for the same inputs. dO [B,Hq,N,d] (p->dtype).
- *   dQ [B,Hq,N,d], dK/dV [B,Hkv,N,d] out (p->dtype; fp32 accumulation).
- *   dS [B,Hq,Nb,Nb] fp32 out: dS[r,c'] = G[r,c'] - g[r,c'] sum_{c<r} G[r,c]
- *   for c' < r and 0 elsewhere, where G[r,c] sums dL/dz over the (r,c) tile.
+/* Gated attention backward (blog section "The Logit Injection Mechanism": the
+ * gradient reaches the scores through the gates inside the softmax).
+ *   O, LSE: outputs of gbs_fwd for the same inputs and p. dO [B,Hq,N,d]
+ *   (p->dtype). dQ [B,Hq,N,d], dK/dV [B,Hkv,N,d] out (p->dtype; fp32
+ *   accumulation). dS [B,Hq,Nb,Nb] fp32 out: dS[r,c'] = G[r,c'] - g[r,c']
+ *   sum_{c in A_r} G[r,c] for c' in A_r and 0 elsewhere, where G[r,c] sums
+ *   dL/dz over the (r,c) tile and A_r is the attended historical set (all of
+ *   c < r in training mode). In sparse and threshold modes (an extension: the
+ *   pages train with every block active) A_r is recomputed from S exactly as
+ *   gbs_fwd selects it, g is renormalised over A_r, and the selection itself
+ *   passes no gradient.
  *   ws: gbs_workspace_bytes(p, GBS_OP_BWD) bytes. */
 GBS_API gbs_status gbs_bwd(const gbs_params* p, const void* Q, const void* K, const void* V,
                    const float* S, const void* O, const float* LSE, const void* dO,

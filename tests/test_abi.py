@@ -89,9 +89,6 @@ def test_threshold_mode_workspace_matches_sparse(lib):
         ps = gb.make_params(2, 8, 2, 4096, 128, 64, 16, "sparse")
         pt = gb.make_params(2, 8, 2, 4096, 128, 64, 16, "threshold", tau=0.05)
         assert gb.workspace_bytes(pt, op) == gb.workspace_bytes(ps, op) > 0
-    pt = gb.make_params(1, 4, 2, 256, 64, 64, 4, "threshold", tau=0.05)
-    ok = ctypes.c_void_p(4096)
-    assert lib.gbs_bwd(ctypes.byref(pt), *([ok] * 12), 1 << 30, None) == 2
 
 
 def test_null_and_misaligned_pointers_rejected(lib):
@@ -114,11 +111,16 @@ def test_workspace_checks(lib):
                        None) == 5
 
 
-def test_backward_requires_training_mode(lib):
-    p = gb.make_params(1, 4, 2, 256, 64, 64, 4, "sparse")
-    ok = ctypes.c_void_p(4096)
-    st = lib.gbs_bwd(ctypes.byref(p), *([ok] * 12), 1 << 30, None)
-    assert st == 2
+def test_sparse_backward_workspace(lib):
+    """Outside training mode the backward also holds K1's lists, the kept-block
+    bitmap and the per-key-tile step lists of the tensor-core path."""
+    pt = gb.make_params(1, 32, 8, 65536, 128, 64, 0, "train")
+    ps = gb.make_params(1, 32, 8, 65536, 128, 64, 64, "sparse")
+    rows, nt = 32 * 1024, 512
+    extra = rows * 64 * 8 + rows * 4 + rows * 32 * 4 + 8 * nt * (1 + 4 * nt) * 4
+    assert gb.workspace_bytes(ps, gb.OP_BWD) >= gb.workspace_bytes(pt, gb.OP_BWD) + extra
+    bad = gb.make_params(1, 4, 2, 256, 64, 64, 4, "threshold", tau=2.0)
+    assert gb.workspace_bytes(bad, gb.OP_BWD) == 0
 
 
 def test_decode_split_bounds(lib):

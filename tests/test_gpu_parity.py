@@ -276,13 +276,15 @@ def test_fwd_sparse_prefill_full_size_sampled(k):
 
 # --------------------------------------------------------------------- backward
 
-def _check_bwd(x, tol, heads=None):
+def _check_bwd(x, tol, heads=None, mode="train", k=0, tau=None):
     d = _dev(x)
-    O, LSE = gb.forward(d["Q"], d["K"], d["V"], d["S"], mode="train")
-    dQ, dK, dV, dS = gb.backward(d["Q"], d["K"], d["V"], d["S"], O, LSE, d["dO"])
+    tv = 0.0 if tau is None else tau
+    O, LSE = gb.forward(d["Q"], d["K"], d["V"], d["S"], mode=mode, topk=k, tau=tv)
+    dQ, dK, dV, dS = gb.backward(d["Q"], d["K"], d["V"], d["S"], O, LSE, d["dO"], mode=mode,
+                                 topk=k, tau=tv)
     torch.cuda.synchronize()
     ref = oracle.gated_attention_backward(np64(x["Q"]), np64(x["K"]), np64(x["V"]), x["S"].numpy(),
-                                          np64(x["dO"]), 64, heads=heads)
+                                          np64(x["dO"]), 64, heads=heads, mode=mode, topk=k, tau=tau)
     errs = {n: rel_err(np64(t) if t.dtype != torch.float32 else t.cpu().numpy().astype(np.float64), r)
             for n, t, r in zip(("dQ", "dK", "dV", "dS"), (dQ, dK, dV, dS), ref[:4])}
     for n, e in errs.items():
@@ -305,6 +307,67 @@ def test_bwd_edge_shapes(shape):
     B, Hq, Hkv, N, d = shape
     for dtype in (torch.bfloat16, torch.float32):
         _check_bwd(_small(3, B, Hq, Hkv, N, d, dtype, scaled=False), TOL_GRAD)
+
+
+# Sparse and threshold backward: gradients through the gates renormalised over
+# the kept blocks; blocks outside A_r get dS = 0.
+
+def test_bwd_sparse_tiny_f32():
+    errs = _check_bwd(make_prefill_inputs(WORKLOADS["tiny_f32_n1024"]), TOL_GRAD, mode="sparse", k=4)
+    assert max(errs.values()) < 1e-4, errs
+
+
+@pytest.mark.parametrize("k", [0, 3, 100])
+@pytest.mark.parametrize("scaled", [True, False])
+def test_bwd_sparse_bf16_small(k, scaled):
+    _check_bwd(_small(13 + k, 1, 8, 2, 1024, 128, torch.bfloat16, scaled), TOL_GRAD,
+               mode="sparse", k=k)
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 2, 64, 128), (2, 4, 4, 320, 64), (1, 4, 1, 448, 128),
+                                   (1, 8, 2, 1344, 64)])
+def test_bwd_sparse_edge_shapes(shape):
+    B, Hq, Hkv, N, d = shape
+    for dtype in (torch.bfloat16, torch.float32):
+        _check_bwd(_small(17, B, Hq, Hkv, N, d, dtype, scaled=False), TOL_GRAD, mode="sparse", k=2)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_bwd_threshold_small(dtype):
+    x = _small(47, 1, 8, 2, 1024, 128, dtype, scaled=True)
+    assert _no_boundary_gates(x["S"], 0.05)
+    _check_bwd(x, TOL_GRAD, mode="threshold", k=6, tau=0.05)
+
+
+def test_bwd_sparse_full_budget_matches_training():
+    x = _dev(_small(53, 1, 4, 2, 512, 128, torch.bfloat16, False))
+    O, LSE = gb.forward(x["Q"], x["K"], x["V"], x["S"], mode="train")
+    gt = gb.backward(x["Q"], x["K"], x["V"], x["S"], O, LSE, x["dO"])
+    gs = gb.backward(x["Q"], x["K"], x["V"], x["S"], O, LSE, x["dO"], mode="sparse", topk=8)
+    torch.cuda.synchronize()
+    for a, b in zip(gt, gs):  # the two normalisers may differ in the last fp32 bit
+        assert rel_err(np64(b), np64(a)) < 1e-2
+
+
+@pytest.mark.parametrize("k", [8, 32])
+def test_bwd_sparse_prefill_full_size_one_group(k):
+    """Planted prefill workload N=65536, 32/8 heads, sparse K, computed in full
+    on the GPU; every gradient of kv-group 0 against the oracle."""
+    w = WORKLOADS["sparse_prefill_bf16_n65536"]
+    x = make_prefill_inputs(w)
+    d = _dev(x)
+    O, LSE = gb.forward(d["Q"], d["K"], d["V"], d["S"], mode="sparse", topk=k)
+    dQ, dK, dV, dS = gb.backward(d["Q"], d["K"], d["V"], d["S"], O, LSE, d["dO"], mode="sparse",
+                                 topk=k)
+    torch.cuda.synchronize()
+    G = w.Hq // w.Hkv
+    ref = oracle.gated_attention_backward(np64(x["Q"][:, :G]), np64(x["K"][:, :1]),
+                                          np64(x["V"][:, :1]), x["S"][:, :G].numpy(),
+                                          np64(x["dO"][:, :G]), 64, mode="sparse", topk=k)
+    got = (dQ[:, :G], dK[:, :1], dV[:, :1], dS[:, :G])
+    for n, t, r in zip(("dQ", "dK", "dV", "dS"), got, ref[:4]):
+        e = rel_err(t.float().cpu().numpy().astype(np.float64), r)
+        assert e < TOL_GRAD, (n, e)
 
 
 def test_bwd_train_full_size_one_group():
