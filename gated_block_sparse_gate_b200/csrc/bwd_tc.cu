@@ -13,8 +13,11 @@
 // dS[r, c'] = G[r, c'] - g[r, c'] sum_{c<r} G[r, c] is formed afterwards from G.
 //
 // Tiling: one CTA per (batch, kv-head, 128-key tile = two 64-key context
-// blocks); K and V stay in shared memory while the CTA walks the G q-heads of
-// the group and every 128-query tile at or after its keys. Per step:
+// blocks); K and V stay in shared memory while the CTA walks a list of the
+// 64-query blocks (of any q-head of the group) that attend its keys, two
+// query blocks per step (query half 0 and 1 of the step's 128 columns; the
+// two may come from different q-heads, and a missing second one is masked). In training mode the list is every query block r >= the
+// tile's first key block, head by head. Per step:
 //   S^T = K Q^T and dP^T = V dO^T   (M=128 keys, N=128 queries, K=d; TMEM)
 //   compute warps: P^T, dZ^T (bf16) back into TMEM, dZ^T into swizzled smem,
 //                  per-warp sums of dZ added into G
@@ -38,11 +41,10 @@
 //
 // Sparse and threshold modes (the gradient through the gates renormalised
 // over the kept blocks A_r; the selection itself passes no gradient) run the
-// same kernel over a step list: bwd_plan_kernel lists, per key tile, the
-// (q-head, query tile) pairs in which some query block keeps one of the tile's
-// two key blocks (plus the diagonal tile), and a compute warp whose (query
-// block, key block) pair is not kept treats it as masked, so its P, dZ and G
-// are 0.
+// same kernel over a list built by bwd_plan_kernel: per key tile, the (q-head,
+// query block) pairs that keep one of the tile's two key blocks or are one of
+// them. A compute warp whose (query block, key block) pair is not kept treats
+// it as masked, so its P, dZ and G are 0.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -113,11 +115,11 @@ struct BwdArgs {
   unsigned int* err;
 };
 
-// Step list of CTA (key tile u, batch x kv-head bk): entry 0 is the count,
-// then (q-head in group << 16 | query tile) for every query tile t >= u of
-// every q-head where some query block of t keeps a key block of u; t = u (the
-// diagonal) always. One warp per CTA (id = u * BKV + bk, the attention
-// kernel's block index), ballot compaction in t order.
+// Query-block list of CTA (key tile u, batch x kv-head bk): entry 0 is the
+// count, then (q-head in group << 16 | query block r) for every r >= 2u of
+// every q-head that keeps key block 2u or 2u + 1, or is one of them (its
+// diagonal block). One warp per CTA (id = u * BKV + bk, the attention
+// kernel's block index), ballot compaction in (q-head, r) order.
 __global__ void bwd_plan_kernel(const uint32_t* __restrict__ mbits, int mwords, int Nb, int n_tiles,
                                 int G, int Hq, int Hkv, int BKV, int32_t* __restrict__ plan,
                                 int plan_stride) {
@@ -127,25 +129,17 @@ __global__ void bwd_plan_kernel(const uint32_t* __restrict__ mbits, int mwords, 
   const int u = id / BKV, bk = id % BKV;
   const int b = bk / Hkv, kvh = bk % Hkv;
   int32_t* out = plan + (size_t)id * plan_stride;
-  const int cw = (2 * u) >> 5, sh = (2 * u) & 31;
+  const int cw = (2 * u) >> 5, sh = (2 * u) & 31;  // key blocks 2u, 2u+1: bits sh, sh+1
   const uint32_t lanes_below = (1u << lane) - 1u;
   int n = 0;
   for (int hh = 0; hh < G; ++hh) {
     const size_t rowbase = (size_t)(b * Hq + kvh * G + hh) * Nb;
-    for (int t0 = u; t0 < n_tiles; t0 += 32) {
-      const int t = t0 + lane;
+    for (int r0 = 2 * u; r0 < Nb; r0 += 32) {
+      const int r = r0 + lane;
       bool need = false;
-      if (t < n_tiles) {
-        if (t == u) {
-          need = true;
-        } else {
-          need = (__ldg(mbits + (rowbase + 2 * t) * mwords + cw) >> sh) & 3u;
-          if (!need && 2 * t + 1 < Nb)
-            need = (__ldg(mbits + (rowbase + 2 * t + 1) * mwords + cw) >> sh) & 3u;
-        }
-      }
+      if (r < Nb) need = r <= 2 * u + 1 || ((__ldg(mbits + (rowbase + r) * mwords + cw) >> sh) & 3u);
       const uint32_t m = __ballot_sync(0xffffffffu, need);
-      if (need) out[1 + n + __popc(m & lanes_below)] = (hh << 16) | t;
+      if (need) out[1 + n + __popc(m & lanes_below)] = (hh << 16) | r;
       n += __popc(m);
     }
   }
@@ -184,19 +178,26 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const int u = (int)(blockIdx.x / BKV);  // key tile; small u = most work, launched first
   const int bk = (int)(blockIdx.x % BKV);
   const int b = bk / p.Hkv, kvh = bk % p.Hkv;
-  const int per_head = a.n_tiles - u;
-  const int32_t* steps = a.plan ? a.plan + (size_t)blockIdx.x * a.plan_stride : nullptr;
-  const int n_steps = steps ? __ldg(steps) : p.G * per_head;
-  // (q-head within the group, query tile) of step j
-  auto step_at = [&](int j, int& hh, int& t) {
-    if (steps) {
-      const int e = __ldg(steps + 1 + j);
-      hh = e >> 16;
-      t = e & 0xffff;
-    } else {
-      hh = j / per_head;
-      t = u + j % per_head;
+  const int per_head = p.Nb - 2 * u;  // training: query blocks r >= 2u of each q-head
+  const int32_t* list = a.plan ? a.plan + (size_t)blockIdx.x * a.plan_stride : nullptr;
+  const int n_entries = list ? __ldg(list) : p.G * per_head;
+  const int n_steps = (n_entries + 1) >> 1;
+  // (batch x q-head row, query block) of list entry i; r = -1 past the end.
+  // Step j takes entries 2j (query half 0) and 2j + 1 (query half 1).
+  auto entry_at = [&](int i, int& bh, int& r) {
+    int hh = 0;
+    r = -1;
+    if (i < n_entries) {
+      if (list) {
+        const int e = __ldg(list + 1 + i);
+        hh = e >> 16;
+        r = e & 0xffff;
+      } else {
+        hh = i / per_head;
+        r = 2 * u + i % per_head;
+      }
     }
+    bh = b * p.Hq + kvh * p.G + hh;
   };
 
   if (threadIdx.x == 0) {
@@ -246,14 +247,16 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const int sj = jj % kQStages;
         if (!mbar_wait(&bars->staged[sj], (jj / kQStages) & 1, abort_flag, a.err, kTimeoutNs))
           return false;
-        int hh, t;
-        step_at(jj, hh, t);
-        const int bh = b * p.Hq + kvh * p.G + hh;
+        int bh0, r0, bh1, r1;
+        entry_at(2 * jj, bh0, r0);
+        entry_at(2 * jj + 1, bh1, r1);
 #pragma unroll 1
         for (int w = 0; w < kComputeWarps; ++w) {
+          // dQ rows of lane quadrant `quad` = query half quad / 2; `hq` = column half of D
           const int quad = w & 3, hq = w >> 2;
-          const int qrow0 = t * kBQ + quad * 32;
-          if (qrow0 >= p.N) continue;
+          const int r = (quad >> 1) ? r1 : r0, bh = (quad >> 1) ? bh1 : bh0;
+          if (r < 0) continue;
+          const int qrow0 = r * 64 + (quad & 1) * 32;
           const uint8_t* stg =
               smem + (hq == 0 ? L::kQOff : L::kdOOff) + sj * L::kTile + quad * (D / 2) * 128;
           for (int bx = 0; bx < D / 64; ++bx)
@@ -274,22 +277,29 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           }
           bulk_wait_group_read0();
         }
-        int hh, t;
-        step_at(j, hh, t);
-        const int bh = b * p.Hq + kvh * p.G + hh;
-        const int q0 = t * kBQ;
-        // rows past the end are never read: a half tile past N is fully masked
-        const int nvalid = (p.N - q0) < kBQ ? (p.N - q0) : kBQ;
+        int bh0, r0, bh1, r1;
+        entry_at(2 * j, bh0, r0);
+        entry_at(2 * j + 1, bh1, r1);
+        const int nv = 1 + (r1 >= 0);  // entry 2j always exists
         float* lse_s = vecs + st * 2 * kBQ;
-        mbar_arrive_expect_tx(&bars->q_full[st], 2 * L::kTile + 2 * nvalid * 4);
+        mbar_arrive_expect_tx(&bars->q_full[st], 2 * L::kTile + nv * 2 * 64 * 4);
         uint8_t* qs = smem + L::kQOff + st * L::kTile;
         uint8_t* ds = smem + L::kdOOff + st * L::kTile;
-        for (int ch = 0; ch < L::kChunks; ++ch) {
-          tma_load_3d(qs + ch * kChunk, &tmQ, &bars->q_full[st], ch * 64, q0, bh);
-          tma_load_3d(ds + ch * kChunk, &tmdO, &bars->q_full[st], ch * 64, q0, bh);
+        for (int h2 = 0; h2 < 2; ++h2) {
+          // a missing query half (only ever half 1) repeats half 0's finite
+          // rows; its warps mask it and its dQ is never reduced
+          const bool own = h2 == 0 || r1 >= 0;
+          const int row = (own && h2 ? r1 : r0) * 64, hd = own && h2 ? bh1 : bh0;
+          for (int ch = 0; ch < L::kChunks; ++ch) {
+            tma_load_3d(qs + ch * kChunk + h2 * (kChunk / 2), &tmQ, &bars->q_full[st], ch * 64, row, hd);
+            tma_load_3d(ds + ch * kChunk + h2 * (kChunk / 2), &tmdO, &bars->q_full[st], ch * 64, row, hd);
+          }
+          if (own) {
+            const size_t off = (size_t)hd * p.N + row;
+            bulk_load(lse_s + h2 * 64, a.LSE + off, 64 * 4, &bars->q_full[st]);
+            bulk_load(lse_s + kBQ + h2 * 64, a.Dvec + off, 64 * 4, &bars->q_full[st]);
+          }
         }
-        bulk_load(lse_s, a.LSE + (size_t)bh * p.N + q0, nvalid * 4, &bars->q_full[st]);
-        bulk_load(lse_s + kBQ, a.Dvec + (size_t)bh * p.N + q0, nvalid * 4, &bars->q_full[st]);
         issued = j + 1;
       }
       if (ok)
@@ -391,14 +401,12 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     bool ok = true;
     for (int j = 0; j < n_steps; ++j) {
       const int st = j % kQStages;
-      int hh, t;
-      step_at(j, hh, t);
-      const int bh = b * p.Hq + kvh * p.G + hh;
-      const int r = 2 * t + hq;  // this warp's query block
+      int bh, r;
+      entry_at(2 * j + hq, bh, r);  // this warp's query block (query half hq)
       const size_t row = (size_t)bh * p.Nb + r;
       int mode = kFull;
       float bias2 = 0.f;
-      if (r >= p.Nb || cj > r) {
+      if (r < 0 || cj >= p.Nb || cj > r) {
         mode = kMasked;
       } else if (cj == r) {
         mode = kCausal;
@@ -618,7 +626,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-bool make_map128(CUtensorMap* m, const void* base, int d, int rows, int heads) {
+bool make_map128(CUtensorMap* m, const void* base, int d, int rows, int heads, int box_rows = 128) {
   static EncodeTiledFn fn = nullptr;
   if (!fn) {
     void* ptr = nullptr;
@@ -631,7 +639,7 @@ bool make_map128(CUtensorMap* m, const void* base, int d, int rows, int heads) {
   }
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)heads};
   const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * rows * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -670,8 +678,8 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, const void* Q, const void* K, con
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap tq, tk, tv, tdo, tdq;
-  if (!make_map128(&tq, Q, D, p.N, p.B * p.Hq) || !make_map128(&tk, K, D, p.N, p.B * p.Hkv) ||
-      !make_map128(&tv, V, D, p.N, p.B * p.Hkv) || !make_map128(&tdo, dO, D, p.N, p.B * p.Hq) ||
+  if (!make_map128(&tq, Q, D, p.N, p.B * p.Hq, 64) || !make_map128(&tk, K, D, p.N, p.B * p.Hkv) ||
+      !make_map128(&tv, V, D, p.N, p.B * p.Hkv) || !make_map128(&tdo, dO, D, p.N, p.B * p.Hq, 64) ||
       !make_map_dq(&tdq, a.dQacc, D, rows))
     return cudaErrorInvalidValue;
   auto kern = bwd_tc_kernel<D>;
@@ -695,13 +703,13 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, const void* Q, const void* K, con
 
 bool bwd_tc_supported(const Problem& p) {
   return p.dtype == GBS_BF16 && p.bs == 64 && (p.d == 64 || p.d == 128) && p.N % 64 == 0 &&
-         (p.Nb + 1) / 2 < 65536;
+         p.Nb <= 65536;
 }
 
 size_t bwd_plan_ints(const Problem& p) {
   if (p.mode == GBS_TRAIN) return 0;
   const size_t n_tiles = (size_t)(p.Nb + 1) / 2;
-  return (size_t)p.B * p.Hkv * n_tiles * (1 + (size_t)p.G * n_tiles);
+  return (size_t)p.B * p.Hkv * n_tiles * (1 + (size_t)p.G * p.Nb);
 }
 
 cudaError_t launch_bwd_tc(const Problem& p, const void* Q, const void* K, const void* V,
@@ -726,7 +734,7 @@ cudaError_t launch_bwd_tc(const Problem& p, const void* Q, const void* K, const 
   a.mbits = sparse ? mbits : nullptr;
   a.mwords = mwords;
   a.plan = sparse ? plan : nullptr;
-  a.plan_stride = 1 + p.G * a.n_tiles;
+  a.plan_stride = 1 + p.G * p.Nb;
   a.err = err;
   if (sparse) {
     const int ctas = p.B * p.Hkv * a.n_tiles;
