@@ -291,43 +291,84 @@ def bench_training_long(dev, peaks, reps=5):
             "bwd_main_ms": bms, "bwd_main_tflops": (fl_fb - fl_f) / bms / 1e9}
 
 
+def _time_backward(gb, Q, K, V, S, O, LSE, dO, mode, k, tau, dev, flush, reps):
+    """Mean whole-call and main-kernel times (ms) of the backward."""
+    pb = gb.make_params(1, Q.shape[1], K.shape[1], Q.shape[2], Q.shape[3], 64, k, mode, Q.dtype,
+                        tau=tau)
+    ws = gb.alloc_workspace(pb, gb.OP_BWD, dev)
+    grads = (torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V), torch.empty_like(S))
+    kw = dict(mode=mode, topk=k, tau=tau, grads=grads, ws=ws)
+    for _ in range(2):
+        gb.backward(Q, K, V, S, O, LSE, dO, **kw)
+    a0, a1, k0, k1 = _events(reps), _events(reps), _events(reps), _events(reps)
+    torch.cuda.synchronize()
+    for i in range(reps):
+        flush.zero_()
+        gb.set_timer(gb.OP_BWD, k0[i], k1[i])
+        a0[i].record()
+        gb.backward(Q, K, V, S, O, LSE, dO, **kw)
+        a1[i].record()
+    torch.cuda.synchronize()
+    gb.set_timer(gb.OP_BWD)
+    gb.check(ws)
+    del ws, grads
+    return (statistics.mean(a.elapsed_time(b) for a, b in zip(a0, a1)),
+            statistics.mean(a.elapsed_time(b) for a, b in zip(k0, k1)))
+
+
 def bench_sparse_prefill(dev, peaks, reps=5):
-    """Sparse prefill N=65536, Top-K sweep; forward only."""
+    """Sparse prefill N=65536: Top-K sweep (forward, and the sparse backward as
+    an extension), and one dynamic-threshold forward (tau=0.01, at most 64)."""
     from gated_block_sparse_gate_b200 import binding as gb
 
     w = WORKLOADS["sparse_prefill_bf16_n65536"]
-    x = make_prefill_inputs(w, with_grad=False)
-    Q, K, V, S = (x[n].to(dev) for n in ("Q", "K", "V", "S"))
+    x = make_prefill_inputs(w)
+    Q, K, V, S, dO = (x[n].to(dev) for n in ("Q", "K", "V", "S", "dO"))
     del x
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     out = {}
-    for k in w.topk:
-        pf = gb.make_params(w.B, w.Hq, w.Hkv, w.N, w.d, w.block, k, "sparse", Q.dtype)
+    cases = [(k, "sparse", 0.0) for k in w.topk] + [(64, "threshold", 0.01)]
+    for k, mode, tau in cases:
+        pf = gb.make_params(w.B, w.Hq, w.Hkv, w.N, w.d, w.block, k, mode, Q.dtype, tau=tau)
         ws = gb.alloc_workspace(pf, gb.OP_FWD, dev)
         O = torch.empty_like(Q)
         LSE = torch.empty(Q.shape[:3], dtype=torch.float32, device=dev)
+        fkw = dict(mode=mode, topk=k, tau=tau, out=O, lse=LSE, ws=ws)
         for _ in range(2):
-            gb.forward(Q, K, V, S, mode="sparse", topk=k, out=O, lse=LSE, ws=ws)
+            gb.forward(Q, K, V, S, **fkw)
         a0, a1, k0, k1 = _events(reps), _events(reps), _events(reps), _events(reps)
         torch.cuda.synchronize()
         for i in range(reps):
             flush.zero_()
             gb.set_timer(gb.OP_FWD, k0[i], k1[i])
             a0[i].record()
-            gb.forward(Q, K, V, S, mode="sparse", topk=k, out=O, lse=LSE, ws=ws)
+            gb.forward(Q, K, V, S, **fkw)
             a1[i].record()
         torch.cuda.synchronize()
         gb.set_timer(gb.OP_FWD)
         gb.check(ws)
         ms = statistics.mean(a.elapsed_time(b) for a, b in zip(a0, a1))
         kms = statistics.mean(a.elapsed_time(b) for a, b in zip(k0, k1))
-        P = sparse_pairs_per_head(w.Nb, w.block, k) * w.B * w.Hq
+        if mode == "sparse":
+            P = sparse_pairs_per_head(w.Nb, w.block, k) * w.B * w.Hq
+        else:  # the kept counts of this S, from K1
+            _, cnt, _, _ = gb.select(S, topk=k, mode=mode, tau=tau)
+            P = int(cnt.sum().item()) * w.block * w.block + w.Nb * w.B * w.Hq * w.block * (w.block + 1) // 2
         fl = 4.0 * w.d * P
         comp_bytes = (Q.numel() * 2 * 2 + K.numel() * 2 * 2 + S.numel() * 4)
         t_roof = max(fl / (peaks["bf16_tflops"] * 1e12), comp_bytes / (peaks["hbm_gbs"] * 1e9))
-        out[f"K{k}"] = {"ms": ms, "tflops": fl / ms / 1e9, "kernel_ms": kms,
-                        "kernel_tflops": fl / kms / 1e9,
-                        "frac_of_roofline": t_roof / (kms * 1e-3)}
+        name = f"K{k}" if mode == "sparse" else f"tau{tau:g}_K{k}"
+        out[name] = {"ms": ms, "tflops": fl / ms / 1e9, "kernel_ms": kms,
+                     "kernel_tflops": fl / kms / 1e9, "frac_of_roofline": t_roof / (kms * 1e-3),
+                     "attended_pairs": P}
+        del ws
+        if mode == "sparse":
+            bms, bkms = _time_backward(gb, Q, K, V, S, O, LSE, dO, mode, k, tau, dev, flush, reps)
+            flb = 10.0 * w.d * P
+            out[name].update({"bwd_ms": bms, "bwd_tflops": flb / bms / 1e9, "bwd_kernel_ms": bkms,
+                              "bwd_kernel_tflops": flb / bkms / 1e9})
+    del Q, K, V, S, dO
+    torch.cuda.empty_cache()
     return out
 
 

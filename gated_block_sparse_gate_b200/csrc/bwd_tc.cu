@@ -163,7 +163,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-              const __grid_constant__ CUtensorMap tmdQ, BwdArgs a) {
+              const __grid_constant__ CUtensorMap tmdQ, const __grid_constant__ CUtensorMap tmQ2,
+              const __grid_constant__ CUtensorMap tmdO2, BwdArgs a) {
   using L = BLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {  // the swizzled tiles need 1024-byte alignment
@@ -235,6 +236,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       prefetch_tmap(&tmV);
       prefetch_tmap(&tmdO);
       prefetch_tmap(&tmdQ);
+      prefetch_tmap(&tmQ2);
+      prefetch_tmap(&tmdO2);
       mbar_arrive_expect_tx(&bars->kv_full, 2 * L::kTile);
       for (int ch = 0; ch < L::kChunks; ++ch) {
         tma_load_3d(smem + L::kKOff + ch * kChunk, &tmK, &bars->kv_full, ch * 64, u * kBK, bk);
@@ -242,14 +245,22 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       }
     }
     if (lane == 0) {
+      // (bh, r) of the two query halves of a step, kept until its dQ is reduced
+      struct Halves {
+        int bh0, r0, bh1, r1;
+      };
+      auto halves_of = [&](int j) {
+        Halves h;
+        entry_at(2 * j, h.bh0, h.r0);
+        entry_at(2 * j + 1, h.bh1, h.r1);
+        return h;
+      };
       // adds step jj's staged dQ (8 warps x 32 rows x D/2 columns) into the accumulator
-      auto reduce_step = [&](int jj) -> bool {
+      auto reduce_step = [&](int jj, const Halves& e) -> bool {
         const int sj = jj % kQStages;
         if (!mbar_wait(&bars->staged[sj], (jj / kQStages) & 1, abort_flag, a.err, kTimeoutNs))
           return false;
-        int bh0, r0, bh1, r1;
-        entry_at(2 * jj, bh0, r0);
-        entry_at(2 * jj + 1, bh1, r1);
+        const int bh0 = e.bh0, r0 = e.r0, bh1 = e.bh1, r1 = e.r1;
 #pragma unroll 1
         for (int w = 0; w < kComputeWarps; ++w) {
           // dQ rows of lane quadrant `quad` = query half quad / 2; `hq` = column half of D
@@ -267,25 +278,35 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       };
       int issued = 0;
       bool ok = true;
+      static_assert(kQStages == 2, "the producer keeps the halves of the last two steps");
+      Halves prev2{0, -1, 0, -1}, prev1{0, -1, 0, -1};
       for (int j = 0; j < n_steps; ++j) {
         const int st = j % kQStages;
+        const Halves cur = halves_of(j);  // list reads overlap the wait below
         // the stage is free once step j-2's MMAs are done and its staged dQ was read
         if (j >= kQStages) {
-          if (!reduce_step(j - kQStages)) {
+          if (!reduce_step(j - kQStages, prev2)) {
             ok = false;
             break;
           }
           bulk_wait_group_read0();
         }
-        int bh0, r0, bh1, r1;
-        entry_at(2 * j, bh0, r0);
-        entry_at(2 * j + 1, bh1, r1);
+        const int bh0 = cur.bh0, r0 = cur.r0, bh1 = cur.bh1, r1 = cur.r1;
         const int nv = 1 + (r1 >= 0);  // entry 2j always exists
         float* lse_s = vecs + st * 2 * kBQ;
         mbar_arrive_expect_tx(&bars->q_full[st], 2 * L::kTile + nv * 2 * 64 * 4);
         uint8_t* qs = smem + L::kQOff + st * L::kTile;
         uint8_t* ds = smem + L::kdOOff + st * L::kTile;
-        for (int h2 = 0; h2 < 2; ++h2) {
+        if (r1 == r0 + 1 && bh1 == bh0) {
+          // two consecutive blocks of one head: 128-row boxes
+          for (int ch = 0; ch < L::kChunks; ++ch) {
+            tma_load_3d(qs + ch * kChunk, &tmQ2, &bars->q_full[st], ch * 64, r0 * 64, bh0);
+            tma_load_3d(ds + ch * kChunk, &tmdO2, &bars->q_full[st], ch * 64, r0 * 64, bh0);
+          }
+          const size_t off = (size_t)bh0 * p.N + r0 * 64;
+          bulk_load(lse_s, a.LSE + off, kBQ * 4, &bars->q_full[st]);
+          bulk_load(lse_s + kBQ, a.Dvec + off, kBQ * 4, &bars->q_full[st]);
+        } else for (int h2 = 0; h2 < 2; ++h2) {
           // a missing query half (only ever half 1) repeats half 0's finite
           // rows; its warps mask it and its dQ is never reduced
           const bool own = h2 == 0 || r1 >= 0;
@@ -301,10 +322,11 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           }
         }
         issued = j + 1;
+        prev2 = prev1;
+        prev1 = cur;
       }
-      if (ok)
-        for (int jj = n_steps - kQStages < 0 ? 0 : n_steps - kQStages; jj < n_steps; ++jj)
-          if (!reduce_step(jj)) break;
+      if (ok && n_steps >= 2) ok = reduce_step(n_steps - 2, prev2);
+      if (ok) reduce_step(n_steps - 1, prev1);
       bulk_wait_group0();  // reductions reach global memory before the CTA exits
       if (*abort_flag) {
         // let loads still in flight land before the CTA exits
@@ -677,9 +699,10 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, const void* Q, const void* K, con
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  CUtensorMap tq, tk, tv, tdo, tdq;
+  CUtensorMap tq, tk, tv, tdo, tdq, tq2, tdo2;
   if (!make_map128(&tq, Q, D, p.N, p.B * p.Hq, 64) || !make_map128(&tk, K, D, p.N, p.B * p.Hkv) ||
       !make_map128(&tv, V, D, p.N, p.B * p.Hkv) || !make_map128(&tdo, dO, D, p.N, p.B * p.Hq, 64) ||
+      !make_map128(&tq2, Q, D, p.N, p.B * p.Hq) || !make_map128(&tdo2, dO, D, p.N, p.B * p.Hq) ||
       !make_map_dq(&tdq, a.dQacc, D, rows))
     return cudaErrorInvalidValue;
   auto kern = bwd_tc_kernel<D>;
@@ -688,7 +711,7 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, const void* Q, const void* K, con
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)(p.B * p.Hkv * a.n_tiles);
   timer_begin(GBS_OP_BWD, st);
-  kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, tdo, tdq, a);
+  kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, tdo, tdq, tq2, tdo2, a);
   timer_end(GBS_OP_BWD, st);
   note_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
