@@ -14,6 +14,7 @@ from .gated_attention import (  # noqa: F401
     gated_attention_forward,
     gated_attention_naive,
     gated_decode,
+    gated_decode_paged,
     log_gates,
     select_blocks,
     threshold_count,

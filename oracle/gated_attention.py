@@ -38,6 +38,9 @@ set H_r = {0..r-1}, attended historical set A_r, q-head h uses kv-head h // G):
          0 elsewhere.
   Decode: one query at position L-1 of a cache of length L; its current block
          is floor((L-1)/bs); A is chosen from the score row S[b, h, :].
+  Paged decode: sequence b's cache is its pages gathered by a block table and
+         cut to its own length L_b, then decoded as above; group-shared
+         selection gives every q-head of a kv group that group's score row.
 
 Options that exist only to pin the oracle against textbook results:
 ``gate="ones"`` replaces every log-gate by 0 (dense causal attention over the
@@ -49,7 +52,9 @@ torch's SDPA; SDPA with an additive mask plus autograd for every gradient
 including dS; central finite differences; gate rows summing to one; dS rows
 summing to zero; shift invariance in S; Top-K against a brute-force rank count;
 full-budget Top-K equal to training mode; a hand-derived closed form; decode
-equal to the last row of sparse prefill; GQA equal to repeated KV heads.
+equal to the last row of sparse prefill; GQA equal to repeated KV heads; paged
+decode equal to contiguous decode under a random page placement and per-length
+truncation; group-shared selection equal to per-head selection on repeated rows.
 No function here is parity-unpinned.
 """
 from __future__ import annotations
@@ -353,6 +358,40 @@ def gated_decode(q, Kc, Vc, S_dec, L, block, topk, scale=None, seqs=None, gate="
             l = np.sum(p)
             O[b, h] = (p / l) @ v
             LSE[b, h] = m + np.log(l)
+    return O, LSE
+
+
+def gated_decode_paged(q, Kpool, Vpool, block_table, seq_lens, S_dec, block, topk, scale=None,
+                       group_shared=False, mode=SPARSE, tau=None, seqs=None):
+    """Decode over a paged, variable-length KV cache: returns (O [B,Hq,d], LSE [B,Hq]).
+
+    A serving-side layout of the decode above (the pages' long-context
+    inference setting; the layout itself is not on the pages): the cache of
+    sequence b is the concatenation of pages Kpool[block_table[b, c]] for its
+    blocks c = 0 .. ceil(L_b / bs) - 1, truncated to its own length
+    L_b = seq_lens[b]; each page holds one context block of every kv head,
+    Kpool [num_pages, Hkv, bs, d]. With ``group_shared`` the G q-heads of a kv
+    group share one score row and so one selection: S_dec is [B, Hkv, Nb] and
+    q-head h reads row h // G. Every sequence is then decoded exactly as
+    gated_decode does it at its own length.
+    """
+    B, Hq, d = q.shape
+    Hkv = Kpool.shape[1]
+    G = Hq // Hkv
+    O = np.full((B, Hq, d), np.nan)
+    LSE = np.full((B, Hq), np.nan)
+    for b in (seqs if seqs is not None else range(B)):
+        L = int(seq_lens[b])
+        nb = -(-L // block)
+        pages = [int(block_table[b, c]) for c in range(nb)]
+        Kc = np.concatenate([_as_f64(Kpool[pg]) for pg in pages], axis=1)[:, :L]
+        Vc = np.concatenate([_as_f64(Vpool[pg]) for pg in pages], axis=1)[:, :L]
+        rows = _as_f64(S_dec[b])
+        if group_shared:
+            rows = np.repeat(rows, G, axis=0)
+        o, lse = gated_decode(q[b:b + 1], Kc[None], Vc[None], rows[None, :, :nb], L, block, topk,
+                              scale=scale, mode=mode, tau=tau)
+        O[b], LSE[b] = o[0], lse[0]
     return O, LSE
 
 

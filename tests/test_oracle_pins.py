@@ -327,6 +327,60 @@ def test_decode_equals_last_prefill_row(L):
     assert rel_err(Od, O[:, :, L - 1]) < 1e-13 and rel_err(Ld, LSE[:, :, L - 1]) < 1e-13
 
 
+def _paged_case(seed, B=3, Hq=4, Hkv=2, d=8, bs=8, Lmax=61):
+    """Contiguous caches, their blocks scattered over a shuffled page pool."""
+    rng = np.random.default_rng(seed)
+    nbmax = -(-Lmax // bs)
+    Kc = rng.standard_normal((B, Hkv, nbmax * bs, d))
+    Vc = rng.standard_normal((B, Hkv, nbmax * bs, d))
+    n_pages = B * nbmax + 5
+    perm = rng.permutation(n_pages)
+    table = perm[:B * nbmax].reshape(B, nbmax)
+    Kpool = rng.standard_normal((n_pages, Hkv, bs, d))  # unused pages hold noise
+    Vpool = rng.standard_normal((n_pages, Hkv, bs, d))
+    for b in range(B):
+        for c in range(nbmax):
+            Kpool[table[b, c]] = Kc[b, :, c * bs:(c + 1) * bs]
+            Vpool[table[b, c]] = Vc[b, :, c * bs:(c + 1) * bs]
+    lens = np.array([Lmax, 17, 40][:B])
+    q = rng.standard_normal((B, Hq, d))
+    return rng, q, Kc, Vc, Kpool, Vpool, table, lens
+
+
+@pytest.mark.parametrize("group_shared", [False, True])
+def test_paged_decode_equals_prefill_row_at_each_length(group_shared):
+    """Each sequence of a paged, variable-length batch equals row L_b - 1 of the
+    naive token-level forward over its own unpaged cache."""
+    rng, q, Kc, Vc, Kpool, Vpool, table, lens = _paged_case(41)
+    B, Hq, d = q.shape
+    Hkv, bs, k = Kc.shape[1], 8, 2
+    nbmax = table.shape[1]
+    S_dec = rng.standard_normal((B, Hkv if group_shared else Hq, nbmax)) * math.sqrt(2)
+    O, LSE = oracle.gated_decode_paged(q, Kpool, Vpool, table, lens, S_dec, bs, k,
+                                       group_shared=group_shared)
+    G = Hq // Hkv
+    for b in range(B):
+        L = int(lens[b])
+        Nb = -(-L // bs)
+        Q = rng.standard_normal((1, Hq, L, d))
+        Q[0, :, L - 1] = q[b]
+        S = rng.standard_normal((1, Hq, Nb, Nb))
+        rows = np.repeat(S_dec[b], G, axis=0) if group_shared else S_dec[b]
+        S[0, :, Nb - 1, :] = rows[:, :Nb]
+        On, Ln, _ = oracle.gated_attention_naive(Q, Kc[b:b + 1, :, :L], Vc[b:b + 1, :, :L], S, bs,
+                                                 mode=oracle.SPARSE, topk=k)
+        assert rel_err(O[b], On[0, :, L - 1]) < 1e-12 and rel_err(LSE[b], Ln[0, :, L - 1]) < 1e-12
+
+
+def test_group_shared_heads_differ_only_by_query():
+    """With one selection per group, heads whose queries are equal get equal outputs."""
+    rng, q, Kc, Vc, Kpool, Vpool, table, lens = _paged_case(43)
+    q[:, 1] = q[:, 0]  # heads 0 and 1 form kv group 0
+    S_dec = rng.standard_normal((3, 2, table.shape[1]))
+    O, LSE = oracle.gated_decode_paged(q, Kpool, Vpool, table, lens, S_dec, 8, 2, group_shared=True)
+    assert np.array_equal(O[:, 0], O[:, 1]) and np.array_equal(LSE[:, 0], LSE[:, 1])
+
+
 def test_attended_pairs_counts():
     S = np.zeros((1, 1, 4, 4))
     # train: history 0+1+2+3 blocks of 4x4 plus 4 triangles of 10
@@ -343,6 +397,15 @@ def _mutant(old, new):
     ns = {"__name__": "oracle_mutant"}
     exec(compile(src.replace(old, new), "<oracle mutant>", "exec"), ns)
     return types.SimpleNamespace(**ns)
+
+
+def test_pins_catch_wrong_page_lookup():
+    bad = _mutant("pages = [int(block_table[b, c]) for c in range(nb)]",
+                  "pages = [c for c in range(nb)]")
+    rng, q, Kc, Vc, Kpool, Vpool, table, lens = _paged_case(47)
+    S_dec = rng.standard_normal((3, 4, table.shape[1]))
+    good = oracle.gated_decode_paged(q, Kpool, Vpool, table, lens, S_dec, 8, 2)[0]
+    assert rel_err(bad.gated_decode_paged(q, Kpool, Vpool, table, lens, S_dec, 8, 2)[0], good) > 1e-3
 
 
 def test_pins_catch_dropped_gate_term():
