@@ -39,6 +39,13 @@ class Params(ctypes.Structure):
                 ("scale", ctypes.c_float), ("tau", ctypes.c_float)]
 
 
+class KvLayout(ctypes.Structure):
+    """gbs_kv_layout: paged / variable-length cache and group-shared selection."""
+    _fields_ = [("block_table", ctypes.c_void_p), ("max_blocks", ctypes.c_int),
+                ("num_pages", ctypes.c_int), ("seq_lens", ctypes.c_void_p),
+                ("group_shared", ctypes.c_int)]
+
+
 _lib = None
 
 
@@ -63,6 +70,8 @@ def load_library(path: str = LIB_PATH):
         "gbs_fwd": (i32, [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "gbs_bwd": (i32, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "gbs_decode": (i32, [P, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]),
+        "gbs_decode_ex": (i32, [P, ctypes.POINTER(KvLayout), vp, vp, vp, vp, vp, vp, i32, vp, sz,
+                                vp]),
         "gbs_set_timer": (i32, [i32, vp, vp]),
         "gbs_launch_count": (ctypes.c_uint64, []),
     }
@@ -179,6 +188,33 @@ def decode(q, Kc, Vc, S, L=None, block=64, topk=32, scale=0.0, num_splits=0, out
         ws = alloc_workspace(p, OP_DECODE, q.device)
     _check(lib.gbs_decode(ctypes.byref(p), _ptr(q), _ptr(Kc), _ptr(Vc), _ptr(S), _ptr(O), _ptr(LSE),
                           num_splits, _ptr(ws), ws.numel(), _stream(stream)), "gbs_decode")
+    return O, LSE
+
+
+def decode_ex(q, Kc, Vc, S, L, block=64, topk=32, scale=0.0, num_splits=0, block_table=None,
+              seq_lens=None, group_shared=False, out=None, lse=None, ws=None, tau=None,
+              stream=None):
+    """gbs_decode_ex: decode over a paged and/or variable-length cache, with one
+    selection per q-head or per kv group. ``L`` is the maximum length; with
+    ``block_table`` (int32 [B, max_blocks]) Kc/Vc are page pools
+    [num_pages, Hkv, block, d]; ``seq_lens`` (int32 [B]) gives each length;
+    with ``group_shared`` S is [B, Hkv, Nb]. Returns (O, LSE)."""
+    lib = load_library()
+    B, Hq, d = q.shape
+    mode = "sparse" if tau is None else "threshold"
+    p = make_params(B, Hq, Kc.shape[1], L, d, block, topk, mode, q.dtype, scale,
+                    0.0 if tau is None else tau)
+    kv = KvLayout(None if block_table is None else block_table.data_ptr(),
+                  0 if block_table is None else block_table.shape[1],
+                  0 if block_table is None else Kc.shape[0],
+                  None if seq_lens is None else seq_lens.data_ptr(), 1 if group_shared else 0)
+    O = out if out is not None else torch.empty_like(q)
+    LSE = lse if lse is not None else torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = alloc_workspace(p, OP_DECODE, q.device)
+    _check(lib.gbs_decode_ex(ctypes.byref(p), ctypes.byref(kv), _ptr(q), _ptr(Kc), _ptr(Vc), _ptr(S),
+                             _ptr(O), _ptr(LSE), num_splits, _ptr(ws), ws.numel(), _stream(stream)),
+           "gbs_decode_ex")
     return O, LSE
 
 

@@ -61,109 +61,158 @@ struct State {
   float m, l, acc[8];
 };
 
-template <typename T, int D>
+// Grid: x = CTA row (one selection row, or a slice of NH q-heads of a
+// group-shared selection row), y = split. Each CTA handles NH q-heads that
+// share one selection and one kv head, so every key and value row it loads
+// serves all NH of them.
+template <typename T, int D, int NH>
 __global__ void __launch_bounds__(kThreads)
 decode_split_kernel(Problem p, const T* __restrict__ q, const T* __restrict__ Kc,
-                    const T* __restrict__ Vc, Selection sel, int cur, int splits,
-                    float* __restrict__ part_ml, float* __restrict__ part_acc) {
+                    const T* __restrict__ Vc, Selection sel, KvLayout kv, int grouped, int n_sub,
+                    int splits, float* __restrict__ part_ml, float* __restrict__ part_acc) {
   constexpr int LPK = D / 8;             // lanes per key row
   constexpr int GPW = 32 / LPK;          // key groups per warp
   constexpr int NGROUPS = (kThreads / 32) * GPW;
   constexpr int ROWS_PER_GROUP = kBS / NGROUPS;
-  __shared__ float s_m[NGROUPS], s_l[NGROUPS];
-  __shared__ float s_acc[NGROUPS][D];
+  __shared__ float s_m[NGROUPS][NH], s_l[NGROUPS][NH];
+  __shared__ float s_acc[NGROUPS][NH][D];
 
-  const int bh = blockIdx.x, split = blockIdx.y;
-  const int b = bh / p.Hq, h = bh % p.Hq, kvh = h / p.G;
+  const int srow = blockIdx.x / n_sub, slice = blockIdx.x % n_sub, split = blockIdx.y;
+  int b, kvh, h0;
+  if (grouped) {
+    b = srow / p.Hkv;
+    kvh = srow % p.Hkv;
+    h0 = kvh * p.G + slice * NH;
+  } else {
+    b = srow / p.Hq;
+    h0 = srow % p.Hq;
+    kvh = h0 / p.G;
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp_in_warp = lane / LPK, sub = lane % LPK;
   const int group = warp * GPW + grp_in_warp;
-  const int n_hist = sel.cnt[bh];
+  int L = p.N;
+  if (kv.seq_lens) {
+    L = __ldg(kv.seq_lens + b);
+    if (L < 1 || L > p.N) {
+      if (threadIdx.x == 0) set_error(kv.err, GBS_ERR_INVALID_ARG);
+      L = L < 1 ? 1 : p.N;
+    }
+  }
+  const int cur = (L - 1) / kBS;
+  const int n_hist = sel.cnt[srow];
   const int n_ent = n_hist + 1;  // + current block
   const int per = (n_ent + splits - 1) / splits;
   const int e0 = split * per, e1 = min(n_ent, e0 + per);
-  const int L = p.N;
 
-  Vec8 qv = load8<T>(q + (size_t)bh * D + sub * 8);
+  Vec8 qv[NH];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) qv.v[i] *= p.scale_log2;
-
-  State st;
-  st.m = -INFINITY;
-  st.l = 0.f;
+  for (int g = 0; g < NH; ++g) {
+    qv[g] = load8<T>(q + ((size_t)b * p.Hq + h0 + g) * D + sub * 8);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) st.acc[i] = 0.f;
+    for (int i = 0; i < 8; ++i) qv[g].v[i] *= p.scale_log2;
+  }
+  State st[NH];
+#pragma unroll
+  for (int g = 0; g < NH; ++g) {
+    st[g].m = -INFINITY;
+    st[g].l = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) st[g].acc[i] = 0.f;
+  }
 
-  const size_t kvbase = ((size_t)(b * p.Hkv + kvh) * L) * D;
+  const size_t contig = ((size_t)(b * p.Hkv + kvh) * p.N) * D;
   for (int e = e0; e < e1; ++e) {
     const bool is_cur = e == n_hist;
-    const int c = is_cur ? cur : sel.idx[(size_t)bh * p.topk + e];
-    const float bias2 = is_cur ? 0.f : sel.logg[(size_t)bh * p.topk + e] * GBS_LOG2E;
+    const int c = is_cur ? cur : sel.idx[(size_t)srow * p.topk + e];
+    const float bias2 = is_cur ? 0.f : sel.logg[(size_t)srow * p.topk + e] * GBS_LOG2E;
+    const int nrows = is_cur ? L - cur * kBS : kBS;  // rows of the block inside the sequence
+    size_t base;  // element offset of the block's first row for this kv head
+    if (kv.btab) {
+      const int page = __ldg(kv.btab + (size_t)b * kv.max_blocks + c);
+      if (page < 0 || page >= kv.num_pages) {  // uniform over the CTA: skip the block
+        if (threadIdx.x == 0) set_error(kv.err, GBS_ERR_INVALID_ARG);
+        continue;
+      }
+      base = (((size_t)page * p.Hkv + kvh) * kBS) * D;
+    } else {
+      base = contig + (size_t)c * kBS * D;
+    }
     // rows handled by this group inside the block
-    const int row0 = c * kBS + group * ROWS_PER_GROUP;
-    Vec8 kv[ROWS_PER_GROUP];
-    float s[ROWS_PER_GROUP];
+    const int row0 = group * ROWS_PER_GROUP;
+    Vec8 kvr[ROWS_PER_GROUP];
+    float s[NH][ROWS_PER_GROUP];
 #pragma unroll
     for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) {
-      const int row = min(row0 + rr, L - 1);
-      kv[rr] = load8<T>(Kc + kvbase + (size_t)row * D + sub * 8);
+      const int row = min(row0 + rr, nrows - 1);
+      kvr[rr] = load8<T>(Kc + base + (size_t)row * D + sub * 8);
     }
 #pragma unroll
     for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) {
-      float d = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) d = fmaf(qv.v[i], kv[rr].v[i], d);
+      for (int g = 0; g < NH; ++g) {
+        float d = 0.f;
 #pragma unroll
-      for (int o = LPK / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-      s[rr] = (row0 + rr < L) ? d + bias2 : -INFINITY;
+        for (int i = 0; i < 8; ++i) d = fmaf(qv[g].v[i], kvr[rr].v[i], d);
+#pragma unroll
+        for (int o = LPK / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+        s[g][rr] = (row0 + rr < nrows) ? d + bias2 : -INFINITY;
+      }
     }
 #pragma unroll
     for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) {
-      const int row = min(row0 + rr, L - 1);
-      kv[rr] = load8<T>(Vc + kvbase + (size_t)row * D + sub * 8);
+      const int row = min(row0 + rr, nrows - 1);
+      kvr[rr] = load8<T>(Vc + base + (size_t)row * D + sub * 8);
     }
-    float mloc = st.m;
 #pragma unroll
-    for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) mloc = fmaxf(mloc, s[rr]);
-    if (mloc > -INFINITY) {
-      const float corr = exp2f(st.m - mloc);
-      st.l *= corr;
+    for (int g = 0; g < NH; ++g) {
+      float mloc = st[g].m;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) st.acc[i] *= corr;
-      st.m = mloc;
+      for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) mloc = fmaxf(mloc, s[g][rr]);
+      if (mloc > -INFINITY) {
+        const float corr = exp2f(st[g].m - mloc);
+        st[g].l *= corr;
 #pragma unroll
-      for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) {
-        const float pr = exp2f(s[rr] - mloc);
-        st.l += pr;
+        for (int i = 0; i < 8; ++i) st[g].acc[i] *= corr;
+        st[g].m = mloc;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) st.acc[i] = fmaf(pr, kv[rr].v[i], st.acc[i]);
+        for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) {
+          const float pr = exp2f(s[g][rr] - mloc);
+          st[g].l += pr;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) st[g].acc[i] = fmaf(pr, kvr[rr].v[i], st[g].acc[i]);
+        }
       }
     }
   }
   // merge the groups of the CTA
-  if (sub == 0) {
-    s_m[group] = st.m;
-    s_l[group] = st.l;
+#pragma unroll
+  for (int g = 0; g < NH; ++g) {
+    if (sub == 0) {
+      s_m[group][g] = st[g].m;
+      s_l[group][g] = st[g].l;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s_acc[group][g][sub * 8 + i] = st[g].acc[i];
   }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) s_acc[group][sub * 8 + i] = st.acc[i];
   __syncthreads();
-  float M = -INFINITY;
+  for (int k = threadIdx.x; k < NH * D; k += kThreads) {
+    const int g = k / D, col = k % D;
+    float M = -INFINITY;
 #pragma unroll
-  for (int g = 0; g < NGROUPS; ++g) M = fmaxf(M, s_m[g]);
-  const size_t pidx = (size_t)bh * splits + split;
-  for (int k = threadIdx.x; k < D; k += kThreads) {
+    for (int gr = 0; gr < NGROUPS; ++gr) M = fmaxf(M, s_m[gr][g]);
     float a = 0.f;
     if (M > -INFINITY)
-      for (int g = 0; g < NGROUPS; ++g) a += s_acc[g][k] * exp2f(s_m[g] - M);
-    part_acc[pidx * D + k] = a;
-  }
-  if (threadIdx.x == 0) {
-    float l = 0.f;
-    if (M > -INFINITY)
-      for (int g = 0; g < NGROUPS; ++g) l += s_l[g] * exp2f(s_m[g] - M);
-    part_ml[pidx * 2] = M;
-    part_ml[pidx * 2 + 1] = l;
+      for (int gr = 0; gr < NGROUPS; ++gr) a += s_acc[gr][g][col] * exp2f(s_m[gr][g] - M);
+    const size_t pidx = ((size_t)b * p.Hq + h0 + g) * splits + split;
+    part_acc[pidx * D + col] = a;
+    if (col == 0) {
+      float l = 0.f;
+      if (M > -INFINITY)
+        for (int gr = 0; gr < NGROUPS; ++gr) l += s_l[gr][g] * exp2f(s_m[gr][g] - M);
+      part_ml[pidx * 2] = M;
+      part_ml[pidx * 2 + 1] = l;
+    }
   }
 }
 
@@ -191,36 +240,58 @@ __global__ void decode_combine_kernel(Problem p, int splits, const float* __rest
   if (threadIdx.x == 0) LSE[bh] = (M + log2f(l)) * GBS_LN2;
 }
 
-template <typename T, int D>
+template <typename T, int D, int NH>
 cudaError_t decode_typed(const Problem& p, const void* q, const void* Kc, const void* Vc,
-                         const Selection& sel, int cur, int splits, float* part_ml,
-                         float* part_acc, void* O, float* LSE, cudaStream_t st) {
-  const int BH = p.B * p.Hq;
+                         const Selection& sel, const KvLayout& kv, bool grouped, int splits,
+                         float* part_ml, float* part_acc, void* O, float* LSE, cudaStream_t st) {
+  const int n_sub = grouped ? p.G / NH : 1;
+  const int rows = grouped ? p.B * p.Hkv * n_sub : p.B * p.Hq;
   timer_begin(GBS_OP_DECODE, st);
-  decode_split_kernel<T, D><<<dim3(BH, splits), kThreads, 0, st>>>(
-      p, (const T*)q, (const T*)Kc, (const T*)Vc, sel, cur, splits, part_ml, part_acc);
+  decode_split_kernel<T, D, NH><<<dim3(rows, splits), kThreads, 0, st>>>(
+      p, (const T*)q, (const T*)Kc, (const T*)Vc, sel, kv, grouped ? 1 : 0, n_sub, splits,
+      part_ml, part_acc);
   timer_end(GBS_OP_DECODE, st);
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  decode_combine_kernel<T, D><<<BH, D, 0, st>>>(p, splits, part_ml, part_acc, (T*)O, LSE);
+  decode_combine_kernel<T, D><<<p.B * p.Hq, D, 0, st>>>(p, splits, part_ml, part_acc, (T*)O, LSE);
   note_launch();
   return cudaGetLastError();
 }
 
+template <typename T, int D>
+cudaError_t decode_heads(const Problem& p, const void* q, const void* Kc, const void* Vc,
+                         const Selection& sel, const KvLayout& kv, bool grouped, int splits,
+                         float* part_ml, float* part_acc, void* O, float* LSE, cudaStream_t st) {
+  const int nh = decode_heads_per_cta(p, grouped);
+  if (nh == 4)
+    return decode_typed<T, D, 4>(p, q, Kc, Vc, sel, kv, grouped, splits, part_ml, part_acc, O, LSE, st);
+  if (nh == 2)
+    return decode_typed<T, D, 2>(p, q, Kc, Vc, sel, kv, grouped, splits, part_ml, part_acc, O, LSE, st);
+  return decode_typed<T, D, 1>(p, q, Kc, Vc, sel, kv, grouped, splits, part_ml, part_acc, O, LSE, st);
+}
+
 }  // namespace
 
+int decode_heads_per_cta(const Problem& p, bool grouped) {
+  if (!grouped) return 1;
+  return p.G % 4 == 0 ? 4 : (p.G % 2 == 0 ? 2 : 1);
+}
+
 cudaError_t launch_decode(const Problem& p, const void* q, const void* Kc, const void* Vc,
-                          const Selection& sel, int cur, int num_splits, float* part_ml,
-                          float* part_acc, void* O, float* LSE, cudaStream_t st) {
+                          const Selection& sel, int num_splits, float* part_ml, float* part_acc,
+                          void* O, float* LSE, cudaStream_t st, const KvLayout& kv, bool grouped) {
   if (p.bs != kBS) return cudaErrorNotSupported;
+#define GBS_DEC(T, DD) \
+  return decode_heads<T, DD>(p, q, Kc, Vc, sel, kv, grouped, num_splits, part_ml, part_acc, O, LSE, st)
   if (p.dtype == GBS_F32) {
-    if (p.d == 64) return decode_typed<float, 64>(p, q, Kc, Vc, sel, cur, num_splits, part_ml, part_acc, O, LSE, st);
-    if (p.d == 128) return decode_typed<float, 128>(p, q, Kc, Vc, sel, cur, num_splits, part_ml, part_acc, O, LSE, st);
+    if (p.d == 64) GBS_DEC(float, 64);
+    if (p.d == 128) GBS_DEC(float, 128);
   } else {
-    if (p.d == 64) return decode_typed<__nv_bfloat16, 64>(p, q, Kc, Vc, sel, cur, num_splits, part_ml, part_acc, O, LSE, st);
-    if (p.d == 128) return decode_typed<__nv_bfloat16, 128>(p, q, Kc, Vc, sel, cur, num_splits, part_ml, part_acc, O, LSE, st);
+    if (p.d == 64) GBS_DEC(__nv_bfloat16, 64);
+    if (p.d == 128) GBS_DEC(__nv_bfloat16, 128);
   }
+#undef GBS_DEC
   return cudaErrorNotSupported;
 }
 

@@ -141,7 +141,8 @@ extern "C" gbs_status gbs_decode_noalloc(const gbs_params* in, const void* q, co
   cudaError_t e = gbs::launch_select(S, (int)rows, pr.Nb, 1, cur, p.topk, pr.mode, pr.log_tau,
                                      sel.idx, sel.cnt, sel.logg, nullptr, st);
   if (e == cudaSuccess)
-    e = gbs::launch_decode(pr, q, Kc, Vc, sel, cur, splits, part_ml, part_acc, O, LSE, st);
+    e = gbs::launch_decode(pr, q, Kc, Vc, sel, splits, part_ml, part_acc, O, LSE, st,
+                           gbs::KvLayout(), false);
   if (e != cudaSuccess) return noalloc_fail(GBS_ERR_CUDA, cudaGetErrorString(e));
   return GBS_OK;
 }

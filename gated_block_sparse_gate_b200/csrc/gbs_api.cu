@@ -333,6 +333,12 @@ gbs_status gbs_bwd(const gbs_params* in, const void* Q, const void* K, const voi
 gbs_status gbs_decode(const gbs_params* in, const void* q, const void* Kc, const void* Vc,
                       const float* S, void* O, float* LSE, int num_splits, void* ws,
                       size_t ws_bytes, void* stream) {
+  return gbs_decode_ex(in, nullptr, q, Kc, Vc, S, O, LSE, num_splits, ws, ws_bytes, stream);
+}
+
+gbs_status gbs_decode_ex(const gbs_params* in, const gbs_kv_layout* kvl, const void* q,
+                         const void* Kc, const void* Vc, const float* S, void* O, float* LSE,
+                         int num_splits, void* ws, size_t ws_bytes, void* stream) {
   g_last_error[0] = 0;
   Problem p;
   gbs_status s = resolve(in, GBS_OP_DECODE, &p);
@@ -342,29 +348,56 @@ gbs_status gbs_decode(const gbs_params* in, const void* q, const void* Kc, const
   if ((s = check_ptrs(6, ptrs, names)) != GBS_OK) return s;
   if (num_splits < 0 || num_splits > kMaxSplits)
     return fail(GBS_ERR_INVALID_ARG, "num_splits %d outside [0, %d]", num_splits, kMaxSplits);
+  KvLayout kv;
+  const bool grouped = kvl && kvl->group_shared;
+  if (kvl) {
+    if (kvl->group_shared != 0 && kvl->group_shared != 1)
+      return fail(GBS_ERR_INVALID_ARG, "group_shared must be 0 or 1");
+    if (kvl->block_table) {
+      if (kvl->max_blocks < p.Nb)
+        return fail(GBS_ERR_INVALID_ARG, "max_blocks (%d) is below ceil(N / block) = %d",
+                    kvl->max_blocks, p.Nb);
+      if (kvl->num_pages <= 0) return fail(GBS_ERR_INVALID_ARG, "num_pages must be positive");
+      if ((uintptr_t)kvl->block_table & 3u)
+        return fail(GBS_ERR_INVALID_ARG, "block_table is not 4-byte aligned");
+    }
+    if (kvl->seq_lens && ((uintptr_t)kvl->seq_lens & 3u))
+      return fail(GBS_ERR_INVALID_ARG, "seq_lens is not 4-byte aligned");
+    kv.btab = kvl->block_table;
+    kv.max_blocks = kvl->max_blocks;
+    kv.num_pages = kvl->num_pages;
+    kv.seq_lens = kvl->seq_lens;
+  }
   DecWs w = carve_dec(p, nullptr);
   if ((s = check_ws(ws, ws_bytes, w.bytes)) != GBS_OK) return s;
   w = carve_dec(p, ws);
+  kv.err = err_word(ws);
   cudaStream_t st = (cudaStream_t)stream;
-  const int BH = p.B * p.Hq;
-  const int cur = (p.N - 1) / p.bs;
-  cudaError_t e = launch_select(S, BH, p.Nb, 1, cur, p.topk, p.mode, p.log_tau, w.sel.idx,
-                                w.sel.cnt, w.sel.logg, nullptr, st);
+  const int sel_rows = grouped ? p.B * p.Hkv : p.B * p.Hq;  // one selection row each
+  const int cur_max = (p.N - 1) / p.bs;
+  SeqLens seq;
+  seq.lens = kv.seq_lens;
+  seq.rows_per_seq = grouped ? p.Hkv : p.Hq;
+  seq.max_len = p.N;
+  cudaError_t e = launch_select(S, sel_rows, p.Nb, 1, kv.seq_lens ? -1 : cur_max, p.topk, p.mode,
+                                p.log_tau, w.sel.idx, w.sel.cnt, w.sel.logg, nullptr, st, nullptr,
+                                nullptr, 0, seq);
   if (e != cudaSuccess) return cuda_status(e, "gbs_decode/select");
-  const int n_ent = (p.topk < cur ? p.topk : cur) + 1;
+  const int n_ent = (p.topk < cur_max ? p.topk : cur_max) + 1;
+  const int cta_rows = grouped ? p.B * p.Hkv * (p.G / decode_heads_per_cta(p, true)) : p.B * p.Hq;
   int splits = num_splits;
   if (splits == 0) {
     // enough CTAs for about two waves of 16 resident 128-thread CTAs per SM
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    splits = (2 * sms * 16 + BH - 1) / BH;
+    splits = (2 * sms * 16 + cta_rows - 1) / cta_rows;
   }
   if (splits > n_ent) splits = n_ent;
   if (splits > kMaxSplits) splits = kMaxSplits;
   if (splits < 1) splits = 1;
-  return cuda_status(launch_decode(p, q, Kc, Vc, w.sel, cur, splits, w.part_ml, w.part_acc, O,
-                                   LSE, st),
+  return cuda_status(launch_decode(p, q, Kc, Vc, w.sel, splits, w.part_ml, w.part_acc, O, LSE, st,
+                                   kv, grouped),
                      "gbs_decode");
 }
 

@@ -40,10 +40,19 @@ struct Selection {
 // threshold modes can also write sel_lse [rows] (the log-sum-exp of S over
 // the kept blocks) and mbits [rows, mwords] (bit c of word c/32 set when block
 // c is kept; every word written).
+// Decode with per-sequence lengths: pass seq_lens [B] (row b holds
+// rows_per_seq consecutive rows; lengths are clamped to [1, max_len]) and
+// decode_cur = -1.
+struct SeqLens {
+  const int32_t* lens = nullptr;
+  int rows_per_seq = 1;
+  int max_len = 0;
+};
 cudaError_t launch_select(const float* S, int n_rows, int row_stride, int rows_per_head,
                           int decode_cur, int topk, int mode, float log_tau, int32_t* idx,
                           int32_t* cnt, float* logg, float* slse, cudaStream_t st,
-                          float* sel_lse = nullptr, uint32_t* mbits = nullptr, int mwords = 0);
+                          float* sel_lse = nullptr, uint32_t* mbits = nullptr, int mwords = 0,
+                          SeqLens seq = SeqLens());
 
 // Exact SIMT path (fp32 math for fp32 or bf16 storage).
 cudaError_t launch_fwd_simt(const Problem& p, const void* Q, const void* K, const void* V,
@@ -55,10 +64,24 @@ cudaError_t launch_bwd_simt(const Problem& p, const void* Q, const void* K, cons
                             float* Dvec, float* Gblk, const uint32_t* mbits, int mwords,
                             cudaStream_t st);
 
-// Decode (split over the selected blocks, then combine).
+// Where the decode finds a sequence's cache: contiguous [B, Hkv, N, d] (btab
+// null) or pages [num_pages, Hkv, 64, d] through btab [B, max_blocks]; every
+// sequence has length N (seq_lens null) or seq_lens[b]. Out-of-range pages or
+// lengths are skipped / clamped on the device and reported in *err.
+struct KvLayout {
+  const int32_t* btab = nullptr;
+  int max_blocks = 0, num_pages = 0;
+  const int32_t* seq_lens = nullptr;
+  unsigned int* err = nullptr;
+};
+
+// Decode (split over the selected blocks, then combine). With `grouped` the
+// selection rows are [B, Hkv] and every q-head of a group uses its group's.
 cudaError_t launch_decode(const Problem& p, const void* q, const void* Kc, const void* Vc,
-                          const Selection& sel, int cur, int num_splits, float* part_ml,
-                          float* part_acc, void* O, float* LSE, cudaStream_t st);
+                          const Selection& sel, int num_splits, float* part_ml, float* part_acc,
+                          void* O, float* LSE, cudaStream_t st, const KvLayout& kv, bool grouped);
+// q-heads one decode CTA serves (they share a selection and a kv head).
+int decode_heads_per_cta(const Problem& p, bool grouped);
 
 // Tensor-core path (sm_100a, bf16). Returns cudaErrorNotSupported when the
 // configuration is outside what the kernel handles.

@@ -82,13 +82,19 @@ __global__ void __launch_bounds__(kWarps * 32)
 select_kernel(const float* __restrict__ S, int n_rows, int row_stride, int rows_per_head,
               int decode_cur, int topk, int mode, float log_tau, int32_t* __restrict__ idx,
               int32_t* __restrict__ cnt, float* __restrict__ logg, float* __restrict__ slse,
-              float* __restrict__ sel_lse, uint32_t* __restrict__ mbits, int mwords) {
+              float* __restrict__ sel_lse, uint32_t* __restrict__ mbits, int mwords,
+              SeqLens seq) {
   __shared__ uint32_t cache_all[kWarps][kRowCache];
   __shared__ uint32_t hist_all[kWarps][256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * kWarps + warp;
   if (row >= n_rows) return;
-  const int r = decode_cur >= 0 ? decode_cur : (row % rows_per_head);
+  int r = decode_cur >= 0 ? decode_cur : (row % rows_per_head);
+  if (seq.lens) {  // decode with one length per sequence: history = its current block
+    int L = __ldg(seq.lens + row / seq.rows_per_seq);
+    L = L < 1 ? 1 : (L > seq.max_len ? seq.max_len : L);
+    r = (L - 1) / 64;
+  }
   const float* srow = S + (size_t)row * row_stride;
   uint32_t* cache = cache_all[warp];
   const bool cached = r <= kRowCache;
@@ -220,12 +226,12 @@ select_kernel(const float* __restrict__ S, int n_rows, int row_stride, int rows_
 cudaError_t launch_select(const float* S, int n_rows, int row_stride, int rows_per_head,
                           int decode_cur, int topk, int mode, float log_tau, int32_t* idx,
                           int32_t* cnt, float* logg, float* slse, cudaStream_t st,
-                          float* sel_lse, uint32_t* mbits, int mwords) {
+                          float* sel_lse, uint32_t* mbits, int mwords, SeqLens seq) {
   if (n_rows <= 0) return cudaSuccess;
   const int grid = (n_rows + kWarps - 1) / kWarps;
   select_kernel<<<grid, kWarps * 32, 0, st>>>(S, n_rows, row_stride, rows_per_head, decode_cur,
                                               topk, mode, log_tau, idx, cnt, logg, slse, sel_lse,
-                                              mbits, mwords);
+                                              mbits, mwords, seq);
   note_launch();
   return cudaGetLastError();
 }

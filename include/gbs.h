@@ -176,6 +176,45 @@ GBS_API gbs_status gbs_decode(const gbs_params* p, const void* q, const void* Kc
                       const float* S, void* O, float* LSE, int num_splits, void* ws,
                       size_t ws_bytes, void* stream);
 
+/* Where gbs_decode_ex finds the KV cache and how the q-heads select (a
+ * serving-side layout of the decode above; the pages describe long-context
+ * inference but no cache layout, so this one is the library's own).
+ *   block_table  NULL: Kc/Vc are contiguous [B, Hkv, L, d] as in gbs_decode.
+ *                Else a DEVICE array [B, max_blocks] of int32: block c of
+ *                sequence b lives in page block_table[b * max_blocks + c], and
+ *                Kc/Vc are page pools [num_pages, Hkv, block, d] (one context
+ *                block of every kv head per page). Only the first
+ *                ceil(L_b / block) entries of a row are read.
+ *   max_blocks   row stride of block_table, >= ceil(p->N / block).
+ *   num_pages    pages in each pool; an entry outside [0, num_pages) is
+ *                skipped on the device and reported by gbs_check as
+ *                GBS_ERR_INVALID_ARG (that sequence's output is then wrong).
+ *   seq_lens     NULL: every sequence has length L = p->N. Else a DEVICE array
+ *                [B] of int32 lengths L_b in [1, p->N] (p->N is the maximum);
+ *                the query of sequence b sits at L_b - 1 and S row entries
+ *                c < (L_b - 1) / block are read. A length outside the range
+ *                is clamped and reported like a bad page.
+ *   group_shared 0: S is [B, Hq, Nb], one selection per q-head (gbs_decode).
+ *                1: S is [B, Hkv, Nb], one selection per kv group, used by its
+ *                Hq / Hkv q-heads, so each selected key/value block is read
+ *                once for the whole group.
+ * All fields are read at call time; the arrays must stay valid until the
+ * call's work on `stream` has finished. */
+typedef struct gbs_kv_layout {
+  const int32_t* block_table;
+  int max_blocks;
+  int num_pages;
+  const int32_t* seq_lens;
+  int group_shared;
+} gbs_kv_layout;
+
+/* gbs_decode over the cache layout `kv` (NULL = gbs_decode). Same workspace
+ * size (gbs_workspace_bytes(p, GBS_OP_DECODE)) and outputs as gbs_decode. */
+GBS_API gbs_status gbs_decode_ex(const gbs_params* p, const gbs_kv_layout* kv, const void* q,
+                                 const void* Kc, const void* Vc, const float* S, void* O,
+                                 float* LSE, int num_splits, void* ws, size_t ws_bytes,
+                                 void* stream);
+
 /* Profiling hook: while `start`/`stop` (cudaEvent_t, caller-owned) are set for
  * `op`, every call of that op records `start` on its stream immediately before
  * its main attention kernel and `stop` immediately after it, so the caller can

@@ -138,3 +138,24 @@ def test_binding_fails_loudly_without_library(tmp_path):
             gb.load_library(str(tmp_path / "missing.so"))
     finally:
         gb._lib = saved
+
+
+@pytest.mark.parametrize("field,value", [("max_blocks", 3), ("num_pages", 0), ("group_shared", 2)])
+def test_decode_ex_layout_checks(lib, field, value):
+    """Paged-layout fields are checked before any launch."""
+    p = gb.make_params(2, 8, 2, 1000, 64, 64, 4, "sparse")  # Nb = 16
+    ok = ctypes.c_void_p(4096)
+    kv = gb.KvLayout(4096, 16, 40, None, 0)
+    setattr(kv, field, value)
+    st = lib.gbs_decode_ex(ctypes.byref(p), ctypes.byref(kv), ok, ok, ok, ok, ok, ok, 0, ok,
+                           1 << 30, None)
+    assert st == 1, lib.gbs_last_error()
+
+
+def test_decode_ex_misaligned_tables(lib):
+    p = gb.make_params(2, 8, 2, 1000, 64, 64, 4, "sparse")
+    ok = ctypes.c_void_p(4096)
+    for kv in (gb.KvLayout(4098, 16, 40, None, 0), gb.KvLayout(None, 0, 0, 4098, 0)):
+        st = lib.gbs_decode_ex(ctypes.byref(p), ctypes.byref(kv), ok, ok, ok, ok, ok, ok, 0, ok,
+                               1 << 30, None)
+        assert st == 1 and b"aligned" in lib.gbs_last_error()
