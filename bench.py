@@ -402,12 +402,60 @@ def bench_decode(dev, peaks, reps=10):
     kv_bytes = w.B * w.Hq * blocks * w.block * w.d * 2 * 2  # K and V per q-head selection
     other = x["q"].numel() * 2 * 2 + x["S"].numel() * 4
     tot = kv_bytes + other
-    del x
+    out = {"ms": ms, "kernel_ms": kms, "tokens_per_s": w.B / (ms * 1e-3),
+           "hbm_gbs": tot / (ms * 1e-3) / 1e9, "kernel_hbm_gbs": kv_bytes / (kms * 1e-3) / 1e9,
+           "frac_of_hbm_roofline": (tot / (peaks["hbm_gbs"] * 1e9)) / (ms * 1e-3),
+           "bytes_per_step": tot}
+
+    def timed(call):
+        for _ in range(3):
+            call()
+        b0, b1, c0, c1 = _events(reps), _events(reps), _events(reps), _events(reps)
+        torch.cuda.synchronize()
+        for i in range(reps):
+            gb.set_timer(gb.OP_DECODE, c0[i], c1[i])
+            b0[i].record()
+            call()
+            b1[i].record()
+        torch.cuda.synchronize()
+        gb.set_timer(gb.OP_DECODE)
+        gb.check(ws)
+        return (statistics.mean(a.elapsed_time(b) for a, b in zip(b0, b1)),
+                statistics.mean(a.elapsed_time(b) for a, b in zip(c0, c1)))
+
+    # one selection per kv group: each selected block is read once per group
+    g = torch.Generator().manual_seed(w.seed + 1)
+    Sg = (torch.randn(w.B, w.Hkv, w.Nb, generator=g) * 2 ** 0.5).to(dev)
+    gms, gkms = timed(lambda: gb.decode_ex(x["q"], x["Kc"], x["Vc"], Sg, w.N, topk=k,
+                                            group_shared=True, out=O, lse=LSE, ws=ws))
+    g_kv = w.B * w.Hkv * blocks * w.block * w.d * 2 * 2
+    g_tot = g_kv + x["q"].numel() * 2 * 2 + Sg.numel() * 4
+    out["group_shared"] = {
+        "ms": gms, "kernel_ms": gkms, "tokens_per_s": w.B / (gms * 1e-3),
+        "hbm_gbs": g_tot / (gms * 1e-3) / 1e9,
+        "frac_of_hbm_roofline": (g_tot / (peaks["hbm_gbs"] * 1e9)) / (gms * 1e-3),
+        "bytes_per_step": g_tot}
+    # the same cache on shuffled 64-token pages through a block table
+    nb = w.N // w.block
+    perm = torch.randperm(w.B * nb, generator=g).to(dev)
+    table = perm.view(w.B, nb).to(torch.int32)
+    pools = []
+    for src in (x["Kc"], x["Vc"]):
+        pool = torch.empty(w.B * nb, w.Hkv, w.block, w.d, dtype=src.dtype, device=dev)
+        pool[perm] = src.view(w.B, w.Hkv, nb, w.block, w.d).permute(0, 2, 1, 3, 4).reshape(
+            w.B * nb, w.Hkv, w.block, w.d)
+        pools.append(pool)
+    del x["Kc"], x["Vc"]
     torch.cuda.empty_cache()
-    return {"ms": ms, "kernel_ms": kms, "tokens_per_s": w.B / (ms * 1e-3),
-            "hbm_gbs": tot / (ms * 1e-3) / 1e9, "kernel_hbm_gbs": kv_bytes / (kms * 1e-3) / 1e9,
-            "frac_of_hbm_roofline": (tot / (peaks["hbm_gbs"] * 1e9)) / (ms * 1e-3),
-            "bytes_per_step": tot}
+    pms, pkms = timed(lambda: gb.decode_ex(x["q"], pools[0], pools[1], x["S"], w.N, topk=k,
+                                            block_table=table, out=O, lse=LSE, ws=ws))
+    out["paged"] = {"ms": pms, "kernel_ms": pkms, "tokens_per_s": w.B / (pms * 1e-3),
+                    "hbm_gbs": tot / (pms * 1e-3) / 1e9,
+                    "frac_of_hbm_roofline": (tot / (peaks["hbm_gbs"] * 1e9)) / (pms * 1e-3),
+                    "bytes_per_step": tot + table.numel() * 4}
+    del x, pools
+    torch.cuda.empty_cache()
+    return out
 
 
 def cpu_baseline_sample(w, budget_s=30.0):

@@ -92,7 +92,7 @@ def test_paged_f32_d64(group_shared):
 
 @pytest.mark.parametrize("Hq,Hkv", [(16, 2), (6, 2), (4, 2), (4, 4)])
 def test_group_shared_group_sizes(Hq, Hkv):
-    """G = 8, 3, 2, 1: four, one, two and one q-heads per CTA."""
+    """G = 8, 3, 2, 1: two, one, two and one q-heads per CTA."""
     x = _paged(11 + Hq, 2, Hq, Hkv, 128, 1500, [1500, 900], torch.bfloat16, True)
     _run_and_check(x, 1500, 4, 2e-2, True)
 
