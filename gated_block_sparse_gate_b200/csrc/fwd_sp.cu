@@ -17,12 +17,16 @@
 // q-heads of one kv group (A, B); each tile walks its own plan one context
 // block (64 keys) per pipeline stage with its own K / V rings, so the tiles
 // never wait for each other's selections, while their MMAs interleave:
-// PV_A(j), S_A(j+1), PV_B(j), S_B(j+1).
+// PV_A(j), S_A(j+1), PV_B(j), S_B(j+1). The gathered key blocks come from all
+// over the history, so their loads are latency-bound: each tile keeps three K
+// slots and two V slots in flight, and K and V have their own producer warps
+// so a V slot waiting for its PV never holds up the next K load.
 // TMEM: S_A (64 columns), S_B (64), O_A (128), O_B (128). P is written back as
 // bf16 over the first 32 columns of its S and read by PV from TMEM.
 // S = Q K^T: M=128, N=64, K=16 per instruction (K-major, 128-byte swizzle);
 // O += P V: A from TMEM, V MN-major.
-// Warps: 0-3 softmax A, 4-7 softmax B, 8 TMA producer, 9 TMEM + MMA issuer.
+// Warps: 0-3 softmax A, 4-7 softmax B, 8 Q/K producer, 9 TMEM + MMA issuer,
+// 10 V producer.
 // Every mbarrier wait is bounded and reports GBS_ERR_TIMEOUT.
 #include <cuda.h>
 
@@ -38,7 +42,10 @@ using namespace sm100;
 
 constexpr int kBM = 128;
 constexpr int kSlot = 64;
-constexpr int kThreads = 320;
+constexpr int kKStages = 3;  // K slots in flight per tile (S needs them first)
+constexpr int kVStages = 2;  // V slots in flight per tile
+constexpr int kKWarp = 8, kMmaWarp = 9, kVWarp = 10;
+constexpr int kThreads = 352;
 constexpr int kTmemCols = 512;
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 constexpr float kRescaleThreshold = 8.0f;
@@ -51,15 +58,16 @@ struct LayoutSp {
   static constexpr int kQTile = kChunks * kQChunk;
   static constexpr int kSlotBytes = kChunks * kSChunk;  // one 64-key K or V block
   static constexpr int kQOff = 0;                           // Q_A, Q_B
-  static constexpr int kKOff = 2 * kQTile;                  // K rings: [tile][2]
-  static constexpr int kVOff = kKOff + 4 * kSlotBytes;      // V rings: [tile][2]
-  static constexpr int kBarOff = kVOff + 4 * kSlotBytes;
+  static constexpr int kKOff = 2 * kQTile;                           // K rings: [tile][3]
+  static constexpr int kVOff = kKOff + 2 * kKStages * kSlotBytes;    // V rings: [tile][2]
+  static constexpr int kBarOff = kVOff + 2 * kVStages * kSlotBytes;
   static constexpr int kSmemBytes = kBarOff + 256;
 };
 
 struct BarsSp {
   uint64_t q_full;
-  uint64_t k_full[2][2], k_empty[2][2], v_full[2][2], v_empty[2][2];  // [tile][stage]
+  uint64_t k_full[2][kKStages], k_empty[2][kKStages];  // [tile][stage]
+  uint64_t v_full[2][kVStages], v_empty[2][kVStages];
   uint64_t s_full[2], p_full[2];
   uint64_t done;
   uint32_t tmem_base;
@@ -131,13 +139,16 @@ fwd_sp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int x = 0; x < 2; ++x)
-      for (int s = 0; s < 2; ++s) {
+    for (int x = 0; x < 2; ++x) {
+      for (int s = 0; s < kKStages; ++s) {
         mbar_init(&bars->k_full[x][s], 1);
         mbar_init(&bars->k_empty[x][s], 1);
+      }
+      for (int s = 0; s < kVStages; ++s) {
         mbar_init(&bars->v_full[x][s], 1);
         mbar_init(&bars->v_empty[x][s], 1);
       }
+    }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bars->s_full[x], 1);
       mbar_init(&bars->p_full[x], 128);
@@ -146,7 +157,7 @@ fwd_sp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     bars->abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -156,11 +167,11 @@ fwd_sp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort_flag = &bars->abort_flag;
 
-  if (warp == 8) {
+  if (warp == kKWarp) {
+    // ------------------------------------------------- Q and K producer (TMA)
     if (lane == 0) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
       mbar_arrive_expect_tx(&bars->q_full, 2 * L::kQTile);
       for (int x = 0; x < 2; ++x)
         for (int ch = 0; ch < L::kChunks; ++ch)
@@ -171,22 +182,47 @@ fwd_sp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       for (int j = 0; ok && j < n_max; ++j) {
         for (int x = 0; ok && x < 2; ++x) {
           if (j >= n[x]) continue;
-          const int st = j & 1;
-          const int c = __ldg(plan[x] + 1 + j);
-          const int ring = x * 2 + st;
-          if (j >= 2 && !mbar_wait(&bars->k_empty[x][st], ((j >> 1) - 1) & 1, abort_flag, a.err, kTimeoutNs)) {
+          const int st = j % kKStages;
+          const int c = __ldg(plan[x] + 1 + j);  // overlaps the wait below
+          // the slot is free once S of step j - kKStages has read it
+          if (j >= kKStages &&
+              !mbar_wait(&bars->k_empty[x][st], (j / kKStages - 1) & 1, abort_flag, a.err, kTimeoutNs)) {
             ok = false;
             break;
           }
-          uint8_t* ks = smem + L::kKOff + ring * L::kSlotBytes;
+          uint8_t* ks = smem + L::kKOff + (x * kKStages + st) * L::kSlotBytes;
           mbar_arrive_expect_tx(&bars->k_full[x][st], L::kSlotBytes);
           for (int ch = 0; ch < L::kChunks; ++ch)
             tma_load_3d(ks + ch * kSChunk, &tmK, &bars->k_full[x][st], ch * 64, c * kSlot, kvz);
-          if (j >= 2 && !mbar_wait(&bars->v_empty[x][st], ((j >> 1) - 1) & 1, abort_flag, a.err, kTimeoutNs)) {
+          issued[x] = j + 1;
+        }
+      }
+      if (*abort_flag) {  // let loads still in flight land before the CTA exits
+        mbar_wait(&bars->q_full, 0, abort_flag, nullptr, 1000000ull);
+        for (int x = 0; x < 2; ++x)
+          for (int j = issued[x] - kKStages < 0 ? 0 : issued[x] - kKStages; j < issued[x]; ++j)
+            mbar_wait(&bars->k_full[x][j % kKStages], (j / kKStages) & 1, abort_flag, nullptr,
+                      1000000ull);
+      }
+    }
+  } else if (warp == kVWarp) {
+    // ------------------------------------------------------ V producer (TMA)
+    if (lane == 0) {
+      prefetch_tmap(&tmV);
+      bool ok = true;
+      int issued[2] = {0, 0};
+      for (int j = 0; ok && j < n_max; ++j) {
+        for (int x = 0; ok && x < 2; ++x) {
+          if (j >= n[x]) continue;
+          const int st = j % kVStages;
+          const int c = __ldg(plan[x] + 1 + j);
+          // the slot is free once PV of step j - kVStages has read it
+          if (j >= kVStages &&
+              !mbar_wait(&bars->v_empty[x][st], (j / kVStages - 1) & 1, abort_flag, a.err, kTimeoutNs)) {
             ok = false;
             break;
           }
-          uint8_t* vs = smem + L::kVOff + ring * L::kSlotBytes;
+          uint8_t* vs = smem + L::kVOff + (x * kVStages + st) * L::kSlotBytes;
           mbar_arrive_expect_tx(&bars->v_full[x][st], L::kSlotBytes);
           for (int ch = 0; ch < L::kChunks; ++ch)
             tma_load_3d(vs + ch * kSChunk, &tmV, &bars->v_full[x][st], ch * 64, c * kSlot, kvz);
@@ -194,24 +230,23 @@ fwd_sp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
       }
       if (*abort_flag) {
-        mbar_wait(&bars->q_full, 0, abort_flag, nullptr, 1000000ull);
         for (int x = 0; x < 2; ++x)
-          for (int j = issued[x] - 2 < 0 ? 0 : issued[x] - 2; j < issued[x]; ++j) {
-            mbar_wait(&bars->k_full[x][j & 1], (j >> 1) & 1, abort_flag, nullptr, 1000000ull);
-            mbar_wait(&bars->v_full[x][j & 1], (j >> 1) & 1, abort_flag, nullptr, 1000000ull);
-          }
+          for (int j = issued[x] - kVStages < 0 ? 0 : issued[x] - kVStages; j < issued[x]; ++j)
+            mbar_wait(&bars->v_full[x][j % kVStages], (j / kVStages) & 1, abort_flag, nullptr,
+                      1000000ull);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(kBM, kSlot, 0);
       constexpr uint32_t idO = idesc_bf16_f32(kBM, D, 1);
       auto issue_s = [&](int x, int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait(&bars->k_full[x][st], (j >> 1) & 1, abort_flag, a.err, kTimeoutNs)) return false;
+        const int st = j % kKStages;
+        if (!mbar_wait(&bars->k_full[x][st], (j / kKStages) & 1, abort_flag, a.err, kTimeoutNs))
+          return false;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(smem + L::kQOff + x * L::kQTile);
-        const uint32_t k_addr = smem_u32(smem + L::kKOff + (x * 2 + st) * L::kSlotBytes);
+        const uint32_t k_addr = smem_u32(smem + L::kKOff + (x * kKStages + st) * L::kSlotBytes);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const int ch = ks >> 2, kk = ks & 3;
@@ -223,11 +258,12 @@ fwd_sp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         return true;
       };
       auto issue_pv = [&](int x, int j) -> bool {
-        const int st = j & 1;
+        const int st = j % kVStages;
         if (!mbar_wait(&bars->p_full[x], j & 1, abort_flag, a.err, kTimeoutNs)) return false;
-        if (!mbar_wait(&bars->v_full[x][st], (j >> 1) & 1, abort_flag, a.err, kTimeoutNs)) return false;
+        if (!mbar_wait(&bars->v_full[x][st], (j / kVStages) & 1, abort_flag, a.err, kTimeoutNs))
+          return false;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(smem + L::kVOff + (x * 2 + st) * L::kSlotBytes);
+        const uint32_t v_addr = smem_u32(smem + L::kVOff + (x * kVStages + st) * L::kSlotBytes);
 #pragma unroll
         for (int ks = 0; ks < kSlot / 16; ++ks)
           mma_ts(tmem + 128 + x * 128, tmem + x * 64 + ks * 8,
@@ -249,7 +285,7 @@ fwd_sp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       mma_commit(&bars->done);
       mbar_wait(&bars->done, 0, abort_flag, a.err, kTimeoutNs);
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------- softmax
     const int x = warp >> 2, quad = warp & 3;
     const int row = quad * 32 + lane;
@@ -358,7 +394,7 @@ fwd_sp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
