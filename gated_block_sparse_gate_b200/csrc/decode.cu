@@ -297,6 +297,23 @@ cudaError_t decode_heads(const Problem& p, const void* q, const void* Kc, const 
 
 }  // namespace
 
+int decode_resident_ctas(const Problem& p, bool grouped) {
+  const int nh = decode_heads_per_cta(p, grouped);
+  const void* fn = nullptr;
+#define GBS_FN(T, DD)                                                                  \
+  fn = nh == 2 ? (const void*)decode_split_kernel<T, DD, 2> : (const void*)decode_split_kernel<T, DD, 1>
+  if (p.dtype == GBS_F32) {
+    if (p.d == 64) GBS_FN(float, 64); else GBS_FN(float, 128);
+  } else {
+    if (p.d == 64) GBS_FN(__nv_bfloat16, 64); else GBS_FN(__nv_bfloat16, 128);
+  }
+#undef GBS_FN
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, kThreads, 0) != cudaSuccess || n < 1)
+    n = 1;
+  return n;
+}
+
 int decode_heads_per_cta(const Problem& p, bool grouped) {
   // Two q-heads per CTA measured fastest on the 64 x 131072 decode with G = 4
   // (0.240 ms against 0.266 ms for one or four): one is the per-head kernel with

@@ -387,11 +387,14 @@ gbs_status gbs_decode_ex(const gbs_params* in, const gbs_kv_layout* kvl, const v
   const int cta_rows = grouped ? p.B * p.Hkv * (p.G / decode_heads_per_cta(p, true)) : p.B * p.Hq;
   int splits = num_splits;
   if (splits == 0) {
-    // enough CTAs for about two waves of 16 resident 128-thread CTAs per SM
+    // enough CTAs for about four waves of the split kernel's resident CTAs
+    // (measured best on the 64 x 131072 decode: 3 splits per q-head row, 2 per
+    // shared-selection row)
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    splits = (2 * sms * 16 + cta_rows - 1) / cta_rows;
+    const int waves_ctas = 4 * sms * decode_resident_ctas(p, grouped);
+    splits = (waves_ctas + cta_rows - 1) / cta_rows;
   }
   if (splits > n_ent) splits = n_ent;
   if (splits > kMaxSplits) splits = kMaxSplits;

@@ -82,6 +82,8 @@ cudaError_t launch_decode(const Problem& p, const void* q, const void* Kc, const
                           void* O, float* LSE, cudaStream_t st, const KvLayout& kv, bool grouped);
 // q-heads one decode CTA serves (they share a selection and a kv head).
 int decode_heads_per_cta(const Problem& p, bool grouped);
+// Decode split CTAs resident per SM for this configuration.
+int decode_resident_ctas(const Problem& p, bool grouped);
 
 // Tensor-core path (sm_100a, bf16). Returns cudaErrorNotSupported when the
 // configuration is outside what the kernel handles.

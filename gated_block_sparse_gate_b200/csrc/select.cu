@@ -221,6 +221,181 @@ select_kernel(const float* __restrict__ S, int n_rows, int row_stride, int rows_
     for (int wi = (base >> 5) + lane; wi < mwords; wi += 32) mbits[(size_t)row * mwords + wi] = 0u;
 }
 
+
+// ------------------------------------------------------------------ decode rows
+// Decode has few score rows (one per sequence and head or kv group) of up to a
+// few thousand blocks, so one CTA of 256 threads takes one row: the row's keys
+// sit in shared memory, the radix passes share one histogram, and the kept
+// blocks are compacted in index order through two block-wide prefix sums (a
+// thread owns a contiguous segment, so the lowest-index ties come first). The
+// selection is the same as select_kernel's.
+constexpr int kRowThreads = 256;
+constexpr int kRowCacheCta = 8192;
+
+__device__ __forceinline__ float key_score(uint32_t u) {
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
+// Block-wide exclusive prefix sum of one int per thread; *total gets the sum.
+__device__ __forceinline__ int block_excl_scan(int v, int* scratch, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  __syncthreads();
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  int wbase = 0, tot = 0;
+  for (int w = 0; w < kRowThreads / 32; ++w) {
+    if (w < warp) wbase += scratch[w];
+    tot += scratch[w];
+  }
+  *total = tot;
+  return wbase + incl - v;
+}
+
+__device__ __forceinline__ float block_max(float v, float* scratch) {
+  v = warp_max(v);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float m = -INFINITY;
+  for (int w = 0; w < kRowThreads / 32; ++w) m = fmaxf(m, scratch[w]);
+  return m;
+}
+
+__device__ __forceinline__ float block_sum(float v, float* scratch) {
+  v = warp_sum(v);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float s = 0.f;
+  for (int w = 0; w < kRowThreads / 32; ++w) s += scratch[w];
+  return s;
+}
+
+__global__ void __launch_bounds__(kRowThreads)
+select_row_cta_kernel(const float* __restrict__ S, int row_stride, int decode_cur, int topk,
+                      int mode, float log_tau, int32_t* __restrict__ idx,
+                      int32_t* __restrict__ cnt, float* __restrict__ logg, SeqLens seq) {
+  __shared__ uint32_t keys[kRowCacheCta];
+  __shared__ uint32_t hist[256];
+  __shared__ int iscr[32];
+  __shared__ float fscr[32];
+  __shared__ int s_bin, s_above;
+  const int row = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int r = decode_cur;
+  if (seq.lens) {
+    int L = __ldg(seq.lens + row / seq.rows_per_seq);
+    L = L < 1 ? 1 : (L > seq.max_len ? seq.max_len : L);
+    r = (L - 1) / 64;
+  }
+  const float* srow = S + (size_t)row * row_stride;
+  for (int c = tid; c < r; c += kRowThreads) keys[c] = ordered_key(__ldg(srow + c));
+  __syncthreads();
+
+  int k = min(topk, r);
+  if (mode == GBS_THRESHOLD && k > 0) {
+    float m = -INFINITY;
+    for (int c = tid; c < r; c += kRowThreads) m = fmaxf(m, key_score(keys[c]));
+    m = block_max(m, fscr);
+    float s = 0.f;
+    for (int c = tid; c < r; c += kRowThreads) s += expf(key_score(keys[c]) - m);
+    const float lse = m + logf(block_sum(s, fscr));
+    int n = 0;
+    for (int c = tid; c < r; c += kRowThreads) n += (key_score(keys[c]) - lse) >= log_tau;
+    int total;
+    block_excl_scan(n, iscr, &total);
+    k = min(k, total);
+  }
+
+  // T = the k-th largest key; need_eq keys equal to T (lowest indices) complete the top k
+  uint32_t T = 0u;
+  int need_eq = 0;
+  if (k > 0 && k < r) {
+    uint32_t prefix = 0u, mask = 0u;
+    int kk = k;
+#pragma unroll 1
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += kRowThreads) hist[i] = 0u;
+      __syncthreads();
+      for (int c = tid; c < r; c += kRowThreads) {
+        const uint32_t u = keys[c];
+        if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      if (warp == 0) {
+        int above;
+        const int bin = find_bin(hist, kk, lane, &above);
+        if (lane == 0) {
+          s_bin = bin;
+          s_above = above;
+        }
+      }
+      __syncthreads();
+      kk -= s_above;
+      prefix |= (uint32_t)s_bin << shift;
+      mask |= 255u << shift;
+    }
+    T = prefix;
+    need_eq = kk;
+  }
+
+  // compaction: thread tid owns blocks [c0, c1) in index order
+  const int seg = (r + kRowThreads - 1) / kRowThreads;
+  const int c0 = min(r, tid * seg), c1 = min(r, c0 + seg);
+  const bool all = k >= r;
+  int gt = 0, eq = 0;
+  if (k > 0 && !all)
+    for (int c = c0; c < c1; ++c) {
+      const uint32_t u = keys[c];
+      gt += u > T;
+      eq += u == T;
+    }
+  int total;
+  const int eq_before = block_excl_scan(eq, iscr, &total);
+  const int eq_quota = k == 0 || all ? 0 : max(0, min(eq, need_eq - eq_before));
+  const int keep = k == 0 ? 0 : (all ? c1 - c0 : gt + eq_quota);
+  int pos = block_excl_scan(keep, iscr, &total);
+  int32_t* out_idx = idx + (size_t)row * topk;
+  float* out_logg = logg + (size_t)row * topk;
+  if (keep > 0) {
+    int eq_seen = 0;
+    for (int c = c0; c < c1; ++c) {
+      const uint32_t u = keys[c];
+      bool kp = all || u > T;
+      if (!all && u == T) {
+        kp = eq_seen < eq_quota;
+        ++eq_seen;
+      }
+      if (kp) {
+        out_idx[pos] = c;
+        out_logg[pos] = key_score(u);  // raw score for now, normalised below
+        ++pos;
+      }
+    }
+  }
+  __syncthreads();  // the kept scores are in global memory, visible to the block
+  float m = -INFINITY;
+  for (int j = tid; j < k; j += kRowThreads) m = fmaxf(m, out_logg[j]);
+  m = block_max(m, fscr);
+  float s = 0.f;
+  for (int j = tid; j < k; j += kRowThreads) s += expf(out_logg[j] - m);
+  const float lse = m + logf(block_sum(s, fscr));
+  for (int j = tid; j < topk; j += kRowThreads) {
+    if (j < k) {
+      out_logg[j] = out_logg[j] - lse;
+    } else {
+      out_idx[j] = -1;
+      out_logg[j] = 0.f;
+    }
+  }
+  if (tid == 0) cnt[row] = k;
+}
+
 }  // namespace
 
 cudaError_t launch_select(const float* S, int n_rows, int row_stride, int rows_per_head,
@@ -228,6 +403,15 @@ cudaError_t launch_select(const float* S, int n_rows, int row_stride, int rows_p
                           int32_t* cnt, float* logg, float* slse, cudaStream_t st,
                           float* sel_lse, uint32_t* mbits, int mwords, SeqLens seq) {
   if (n_rows <= 0) return cudaSuccess;
+  // decode rows (one history length per row, outputs idx/cnt/logg only): one CTA per row
+  const bool decode = decode_cur >= 0 || seq.lens;
+  const int r_max = seq.lens ? (seq.max_len - 1) / 64 : decode_cur;
+  if (decode && mode != GBS_TRAIN && !slse && !sel_lse && !mbits && r_max <= kRowCacheCta) {
+    select_row_cta_kernel<<<n_rows, kRowThreads, 0, st>>>(S, row_stride, decode_cur, topk, mode,
+                                                          log_tau, idx, cnt, logg, seq);
+    note_launch();
+    return cudaGetLastError();
+  }
   const int grid = (n_rows + kWarps - 1) / kWarps;
   select_kernel<<<grid, kWarps * 32, 0, st>>>(S, n_rows, row_stride, rows_per_head, decode_cur,
                                               topk, mode, log_tau, idx, cnt, logg, slse, sel_lse,

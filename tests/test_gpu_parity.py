@@ -427,3 +427,28 @@ def test_decode_full_size_sampled():
     _check_decode(x, w.N, 32, TOL_BF16, seqs=[0, 37, 63])
     del x
     torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------------ determinism
+
+def test_run_to_run_determinism():
+    """Forward and decode have no atomics: their outputs repeat bit for bit.
+    In the backward dK and dV accumulate inside one CTA (bitwise too); dQ and the
+    tile sums behind dS are summed across CTAs in hardware order, so they repeat
+    to within fp32 rounding."""
+    x = _dev(_small(61, 1, 8, 2, 1024, 128, torch.bfloat16, scaled=False))
+    for mode, k in (("train", 0), ("sparse", 3)):
+        O1, L1 = gb.forward(x["Q"], x["K"], x["V"], x["S"], mode=mode, topk=k)
+        O2, L2 = gb.forward(x["Q"], x["K"], x["V"], x["S"], mode=mode, topk=k)
+        assert torch.equal(O1, O2) and torch.equal(L1, L2), mode
+        g1 = gb.backward(x["Q"], x["K"], x["V"], x["S"], O1, L1, x["dO"], mode=mode, topk=k)
+        g2 = gb.backward(x["Q"], x["K"], x["V"], x["S"], O1, L1, x["dO"], mode=mode, topk=k)
+        assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2]), mode
+        for a, b in ((g1[0], g2[0]), (g1[3], g2[3])):
+            assert rel_err(np64(a), np64(b)) < 1e-5, mode
+    from dataclasses import replace
+    w = replace(WORKLOADS["sparse_decode_bf16_b64_l131072"], B=4, N=5000)
+    d = {n: t.to(DEV) for n, t in make_decode_inputs(w, B=4, L=5000).items()}
+    r1 = gb.decode(d["q"], d["Kc"], d["Vc"], d["S"], topk=16)
+    r2 = gb.decode(d["q"], d["Kc"], d["Vc"], d["S"], topk=16)
+    assert torch.equal(r1[0], r2[0]) and torch.equal(r1[1], r2[1])
