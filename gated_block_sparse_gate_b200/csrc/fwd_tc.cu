@@ -94,6 +94,20 @@ struct FwdArgs {
   unsigned int* err;
 };
 
+enum : int { kMasked = 0, kDiag = 1, kFull = 2 };
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -272,32 +286,49 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_stages; ++j) {
-      const float bias0 = slot_bias(a, plan_tile, bh, j, 0, half, myr);
-      const float bias1 = slot_bias(a, plan_tile, bh, j, 1, half, myr);
+      // per slot: +inf = causal current block, -inf = masked, else the log2 gate
+      const float sb0 = slot_bias(a, plan_tile, bh, j, 0, half, myr);
+      const float sb1 = slot_bias(a, plan_tile, bh, j, 1, half, myr);
+      const int kind[2] = {sb0 == INFINITY ? kDiag : (sb0 == -INFINITY ? kMasked : kFull),
+                           sb1 == INFINITY ? kDiag : (sb1 == -INFINITY ? kMasked : kFull)};
+      const float bias[2] = {kind[0] == kFull ? sb0 : 0.f, kind[1] == kFull ? sb1 : 0.f};
       if (!mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1, abort_flag, a.err, kTimeoutNs)) {
         ok = false;
         break;
       }
       tc_fence_after();
       const uint32_t tS = tmem + lane_off + (j & 1) * 128;
-      uint32_t raw[4][32];
+      // pass 1: per-slot maximum of the scaled, biased logits; slot 1 stays in
+      // registers, slot 0 is read again in pass 2 (keeps register use low)
+      uint32_t v1[64];
+      float smax[2];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, raw[q]);
-      tmem_wait_ld();
-      float v[128];
-      float mx = -INFINITY;
+      for (int s = 0; s < 2; ++s) {
+        uint32_t v[64];
+        tmem_ld32(tS + s * 64, *reinterpret_cast<uint32_t(*)[32]>(v));
+        tmem_ld32(tS + s * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+        tmem_wait_ld();
+        if (kind[s] == kDiag) {
 #pragma unroll
-      for (int k = 0; k < 128; ++k) {
-        const float bias = k < 64 ? bias0 : bias1;
-        const int kl = k & 63;
-        float x = __uint_as_float(raw[k >> 5][k & 31]);
-        if (bias == INFINITY)
-          x = kl <= iloc ? x * sc : -INFINITY;
-        else
-          x = bias == -INFINITY ? -INFINITY : fmaf(x, sc, bias);
-        v[k] = x;
-        mx = fmaxf(mx, x);
+          for (int k = 0; k < 64; ++k)
+            if (k > iloc) v[k] = __float_as_uint(-INFINITY);
+        }
+        float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < 64; k += 8) {
+          a0 = max3(a0, __uint_as_float(v[k]), __uint_as_float(v[k + 1]));
+          a1 = max3(a1, __uint_as_float(v[k + 2]), __uint_as_float(v[k + 3]));
+          a2 = max3(a2, __uint_as_float(v[k + 4]), __uint_as_float(v[k + 5]));
+          a3 = max3(a3, __uint_as_float(v[k + 6]), __uint_as_float(v[k + 7]));
+        }
+        const float rawmax = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+        smax[s] = kind[s] == kMasked ? -INFINITY : fmaf(rawmax, sc, bias[s]);
+        if (s == 1) {
+#pragma unroll
+          for (int k = 0; k < 64; ++k) v1[k] = v[k];
+        }
       }
+      const float mx = fmaxf(smax[0], smax[1]);
       const bool need = mx > m + kRescaleThreshold;
       // PV of the previous stage must be complete before O is touched; waiting
       // every stage also keeps the o_done parity unambiguous.
@@ -320,22 +351,74 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
           for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
           tmem_st32(tO + q * 32, o);
         }
-        l *= f;
+        if (need) l *= f;
       }
       if (need) m = mx;
       const float mu = m == -INFINITY ? 0.f : m;
-      uint32_t pk[2][32];
-      float ls = 0.f;
+      float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+      // pass 2, slot 0: 32-column chunks; bf16 P of keys [32c, 32c+32) goes to
+      // columns [16c, 16c+16), which this pass has already read
 #pragma unroll
-      for (int k = 0; k < 64; ++k) {
-        const float p0 = ex2(v[2 * k] - mu), p1 = ex2(v[2 * k + 1] - mu);
-        ls += p0 + p1;
-        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-        pk[k >> 5][k & 31] = *reinterpret_cast<const uint32_t*>(&pb);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[16];
+        if (kind[0] == kMasked) {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) pk[k] = 0u;
+        } else {
+          uint32_t v[32];
+          tmem_ld32(tS + c * 32, v);
+          tmem_wait_ld();
+          const float cst = bias[0] - mu;
+#pragma unroll
+          for (int k = 0; k < 32; k += 4) {
+            float x0 = fmaf(__uint_as_float(v[k]), sc, cst);
+            float x1 = fmaf(__uint_as_float(v[k + 1]), sc, cst);
+            float x2 = fmaf(__uint_as_float(v[k + 2]), sc, cst);
+            float x3 = fmaf(__uint_as_float(v[k + 3]), sc, cst);
+            if (kind[0] == kDiag) {
+              const int kk = c * 32 + k;
+              if (kk > iloc) x0 = -INFINITY;
+              if (kk + 1 > iloc) x1 = -INFINITY;
+              if (kk + 2 > iloc) x2 = -INFINITY;
+              if (kk + 3 > iloc) x3 = -INFINITY;
+            }
+            const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+            l0 += p0;
+            l1 += p1;
+            l2 += p2;
+            l3 += p3;
+            pk[k / 2] = cvt_bf16x2(p0, p1);
+            pk[k / 2 + 1] = cvt_bf16x2(p2, p3);
+          }
+        }
+        tmem_st16(tS + c * 16, pk);
       }
-      l += ls;
-      tmem_st32(tS, pk[0]);
-      tmem_st32(tS + 32, pk[1]);
+      // slot 1 from registers -> columns [32, 64) (slot 0's upper half, read above)
+      {
+        uint32_t pk[32];
+        if (kind[1] == kMasked) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) pk[k] = 0u;
+        } else {
+          const float cst = bias[1] - mu;
+#pragma unroll
+          for (int k = 0; k < 64; k += 4) {
+            // pass 1 already set the causal mask's -inf in v1
+            const float p0 = ex2(fmaf(__uint_as_float(v1[k]), sc, cst));
+            const float p1 = ex2(fmaf(__uint_as_float(v1[k + 1]), sc, cst));
+            const float p2 = ex2(fmaf(__uint_as_float(v1[k + 2]), sc, cst));
+            const float p3 = ex2(fmaf(__uint_as_float(v1[k + 3]), sc, cst));
+            l0 += p0;
+            l1 += p1;
+            l2 += p2;
+            l3 += p3;
+            pk[k / 2] = cvt_bf16x2(p0, p1);
+            pk[k / 2 + 1] = cvt_bf16x2(p2, p3);
+          }
+        }
+        tmem_st32(tS + 32, pk);
+      }
+      l += (l0 + l1) + (l2 + l3);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p_full[j & 1]);
