@@ -281,10 +281,6 @@ gbs_status gbs_fwd(const gbs_params* in, const void* Q, const void* K, const voi
     e = launch_fwd_tc2(p, Q, K, V, S, w.sel.slse, O, LSE, err_word(ws), st);
     if (e != cudaErrorNotSupported) return cuda_status(e, "gbs_fwd/attention");
   }
-  if (fwd_sp_supported(p)) {
-    e = launch_fwd_sp(p, Q, K, V, w.sel, w.plan, (int)plan_stride(p), O, LSE, err_word(ws), st);
-    if (e != cudaErrorNotSupported) return cuda_status(e, "gbs_fwd/attention");
-  }
   if (p.dtype == GBS_BF16 && fwd_tc_supported(p)) {
     e = launch_fwd_tc(p, Q, K, V, S, w.sel, w.plan, (int)plan_stride(p), O, LSE, err_word(ws), st);
     if (e != cudaErrorNotSupported) return cuda_status(e, "gbs_fwd/attention");

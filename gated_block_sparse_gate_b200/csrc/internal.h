@@ -101,12 +101,6 @@ bool fwd_tc2_supported(const Problem& p);
 // two query blocks' Top-K lists plus their current blocks, with per-half biases).
 cudaError_t launch_plan(const Problem& p, const Selection& sel, int32_t* plan, int plan_stride,
                         int n_tiles, cudaStream_t st);
-// Sparse mode, even q-heads-per-kv-head ratio: two query tiles per CTA, one
-// context block per pipeline stage.
-cudaError_t launch_fwd_sp(const Problem& p, const void* Q, const void* K, const void* V,
-                          const Selection& sel, int32_t* plan, int plan_stride, void* O,
-                          float* LSE, unsigned int* err, cudaStream_t st);
-bool fwd_sp_supported(const Problem& p);
 // Backward. `slse` is the gate normaliser (over H_r in training mode, over the
 // kept blocks otherwise); outside training mode `mbits` is K1's kept-block
 // bitmap and `plan` a workspace of bwd_plan_ints(p) ints where the launcher
