@@ -71,9 +71,10 @@ struct State {
 // Grid: x = CTA row (one selection row, or a slice of NH q-heads of a
 // group-shared selection row), y = split. Each CTA handles NH q-heads that
 // share one selection and one kv head, so every key and value row it loads
-// serves all NH of them.
+// serves all NH of them. With NH = 2 the registers are capped for four CTAs
+// per SM (no spills), which keeps enough rows in flight.
 template <typename T, int D, int NH>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, NH == 2 ? 4 : 1)
 decode_split_kernel(Problem p, const T* __restrict__ q, const T* __restrict__ Kc,
                     const T* __restrict__ Vc, Selection sel, KvLayout kv, int grouped, int n_sub,
                     int splits, float* __restrict__ part_ml, float* __restrict__ part_acc) {
