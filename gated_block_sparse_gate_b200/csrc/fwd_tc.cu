@@ -54,7 +54,6 @@ using namespace sm100;
 constexpr int kBM = 128;            // query rows per tile
 constexpr int kSlot = 64;           // keys per slot (one context block)
 constexpr int kBN = 2 * kSlot;      // keys per stage
-constexpr int kStages = 1;
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 256;  // two CTAs per SM share the 512 columns
 constexpr uint64_t kTimeoutNs = 4000000000ull;
@@ -69,19 +68,18 @@ struct Layout {
   static constexpr int kKVBytes = kChunks * kKVChunk;      // per stage, per tensor
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kQBytes;
-  static constexpr int kVOff = kKOff + kStages * kKVBytes;
-  static constexpr int kBarOff = kVOff + kStages * kKVBytes;
+  static constexpr int kVOff = kKOff + kKVBytes;   // one K and one V stage
+  static constexpr int kBarOff = kVOff + kKVBytes;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers + alignment slack
 };
 
 struct Barriers {
   uint64_t q_full;
-  uint64_t k_full[kStages];
-  uint64_t v_full[kStages];
+  uint64_t k_full;
+  uint64_t v_full;
   uint64_t k_empty, v_empty;
   uint64_t s_full;
   uint64_t p_full;
-  uint64_t o_done;
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -165,15 +163,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars->k_full[s], 1);
-      mbar_init(&bars->v_full[s], 1);
-    }
+    mbar_init(&bars->k_full, 1);
+    mbar_init(&bars->v_full, 1);
     mbar_init(&bars->k_empty, 1);
     mbar_init(&bars->v_empty, 1);
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->p_full, 128);
-    mbar_init(&bars->o_done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     fence_barrier_init();
@@ -207,18 +202,18 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         uint8_t* vst = smem + L::kVOff;
         // K is free once S of the previous stage has read it
         if (j > 0 && !mbar_wait(&bars->k_empty, (j - 1) & 1, abort_flag, a.err, kTimeoutNs)) break;
-        mbar_arrive_expect_tx(&bars->k_full[0], L::kKVBytes);
+        mbar_arrive_expect_tx(&bars->k_full, L::kKVBytes);
         for (int ch = 0; ch < L::kChunks; ++ch) {
-          tma_load_3d(kst + ch * L::kKVChunk, &tmK, &bars->k_full[0], ch * 64, c0 * kSlot, kvz);
-          tma_load_3d(kst + ch * L::kKVChunk + kSlotBytes, &tmK, &bars->k_full[0], ch * 64,
+          tma_load_3d(kst + ch * L::kKVChunk, &tmK, &bars->k_full, ch * 64, c0 * kSlot, kvz);
+          tma_load_3d(kst + ch * L::kKVChunk + kSlotBytes, &tmK, &bars->k_full, ch * 64,
                       c1 * kSlot, kvz);
         }
         // V is free once PV of the previous stage has read it
         if (j > 0 && !mbar_wait(&bars->v_empty, (j - 1) & 1, abort_flag, a.err, kTimeoutNs)) break;
-        mbar_arrive_expect_tx(&bars->v_full[0], L::kKVBytes);
+        mbar_arrive_expect_tx(&bars->v_full, L::kKVBytes);
         for (int ch = 0; ch < L::kChunks; ++ch) {
-          tma_load_3d(vst + ch * L::kKVChunk, &tmV, &bars->v_full[0], ch * 64, c0 * kSlot, kvz);
-          tma_load_3d(vst + ch * L::kKVChunk + kSlotBytes, &tmV, &bars->v_full[0], ch * 64,
+          tma_load_3d(vst + ch * L::kKVChunk, &tmV, &bars->v_full, ch * 64, c0 * kSlot, kvz);
+          tma_load_3d(vst + ch * L::kKVChunk + kSlotBytes, &tmV, &bars->v_full, ch * 64,
                       c1 * kSlot, kvz);
         }
         issued = j + 1;
@@ -226,8 +221,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       if (*abort_flag) {
         mbar_wait(&bars->q_full, 0, abort_flag, nullptr, 1000000ull);
         if (issued > 0) {
-          mbar_wait(&bars->k_full[0], (issued - 1) & 1, abort_flag, nullptr, 1000000ull);
-          mbar_wait(&bars->v_full[0], (issued - 1) & 1, abort_flag, nullptr, 1000000ull);
+          mbar_wait(&bars->k_full, (issued - 1) & 1, abort_flag, nullptr, 1000000ull);
+          mbar_wait(&bars->v_full, (issued - 1) & 1, abort_flag, nullptr, 1000000ull);
         }
       }
     }
@@ -242,7 +237,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       bool ok = mbar_wait(&bars->q_full, 0, abort_flag, a.err, kTimeoutNs);
       for (int j = 0; ok && j < n_stages; ++j) {
         // S_j = Q K_j^T (after PV_{j-1} has read P_{j-1} from the same columns)
-        if (!mbar_wait(&bars->k_full[0], j & 1, abort_flag, a.err, kTimeoutNs)) break;
+        if (!mbar_wait(&bars->k_full, j & 1, abort_flag, a.err, kTimeoutNs)) break;
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
@@ -254,7 +249,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mma_commit(&bars->k_empty);
         // O += P_j V_j
         if (!mbar_wait(&bars->p_full, j & 1, abort_flag, a.err, kTimeoutNs) ||
-            !mbar_wait(&bars->v_full[0], j & 1, abort_flag, a.err, kTimeoutNs))
+            !mbar_wait(&bars->v_full, j & 1, abort_flag, a.err, kTimeoutNs))
           break;
         tc_fence_after();
 #pragma unroll
