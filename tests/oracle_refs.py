@@ -14,8 +14,11 @@ import torch
 import torch.nn.functional as F
 
 
-def _selection_mask(S, Nb, mode, topk):
-    """bool [B,H,Nb,Nb]: key block c attended as history by query block r."""
+def _selection_mask(S, Nb, mode, topk, tau=None):
+    """bool [B,H,Nb,Nb]: key block c attended as history by query block r.
+
+    Threshold mode keeps, of the blocks whose gate over the whole history
+    (torch.softmax of the row) reaches tau, the topk with the largest scores."""
     B, H = S.shape[:2]
     r = torch.arange(Nb)[:, None]
     c = torch.arange(Nb)[None, :]
@@ -27,6 +30,9 @@ def _selection_mask(S, Nb, mode, topk):
         for h in range(H):
             for rr in range(1, Nb):
                 k = min(topk, rr)
+                if mode == "threshold":
+                    gates = torch.softmax(S[b, h, rr, :rr].detach(), dim=0)
+                    k = min(k, int((gates >= tau).sum()))
                 if k:
                     top = torch.topk(S[b, h, rr, :rr].detach(), k).indices
                     sel[b, h, rr, top] = True
@@ -34,7 +40,7 @@ def _selection_mask(S, Nb, mode, topk):
 
 
 def sdpa_gated(Q, K, V, S, block, mode="train", topk=None, scale=None, renormalise=True,
-               dO=None, gate="log_softmax"):
+               dO=None, gate="log_softmax", tau=None):
     """(O, LSE, dQ, dK, dV, dS) from SDPA + additive mask + autograd, float64."""
     Q = torch.as_tensor(np.asarray(Q, dtype=np.float64)).requires_grad_(True)
     K = torch.as_tensor(np.asarray(K, dtype=np.float64)).requires_grad_(True)
@@ -45,7 +51,7 @@ def sdpa_gated(Q, K, V, S, block, mode="train", topk=None, scale=None, renormali
     Nb = S.shape[2]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    sel, hist = _selection_mask(S, Nb, mode, topk)
+    sel, hist = _selection_mask(S, Nb, mode, topk, tau)
     norm_set = sel if renormalise else hist
     ls = torch.log_softmax(S.masked_fill(~norm_set, -1e300), dim=-1)
     if gate == "ones":

@@ -129,6 +129,25 @@ def test_sparse_matches_sdpa_autograd(topk, renormalise):
         assert rel_err(x, ref[name]) < 1e-9, name
 
 
+@pytest.mark.parametrize("tau,topk", [(0.05, 3), (0.15, 8), (0.3, 5)])
+def test_threshold_matches_sdpa_autograd(tau, topk):
+    """Threshold selection (gate over the whole history >= tau, at most topk
+    blocks) with gates renormalised over the kept set: forward and all four
+    gradients against SDPA + autograd with the mask built by torch."""
+    B, Hq, Hkv, N, d, bs = 1, 4, 2, 160, 8, 16
+    Q, K, V, S, dO = _rand(40 + topk, B, Hq, Hkv, N, d, bs)
+    kw = dict(mode=oracle.THRESHOLD, topk=topk, tau=tau)
+    O, LSE = oracle.gated_attention_forward(Q, K, V, S, bs, **kw)
+    dQ, dK, dV, dS, _ = oracle.gated_attention_backward(Q, K, V, S, dO, bs, **kw)
+    ref = sdpa_gated(Q, K, V, S, bs, mode="threshold", topk=topk, tau=tau, dO=dO)
+    for name, x in dict(O=O, LSE=LSE, dQ=dQ, dK=dK, dV=dV, dS=dS).items():
+        assert rel_err(x, ref[name]) < 1e-9, name
+    # the threshold must bind on some rows and the budget on others
+    _, cnt, _, _ = oracle.select_blocks(S, N // bs, topk, mode=oracle.THRESHOLD, tau=tau)
+    r = np.arange(N // bs)
+    assert (cnt < np.minimum(topk, r)).any()
+
+
 # ---------------------------------------------------------- finite differences
 
 def _fd_check(Q, K, V, S, bs, W, n_pick=24, seed=0, eps=1e-6, bwd=None):
