@@ -146,6 +146,9 @@ gbs_status resolve(const gbs_params* in, int op, Problem* out) {
   const size_t Nb = ((size_t)q.N + q.block - 1) / q.block;
   if ((size_t)q.B * q.Hq * Nb * Nb > ((size_t)1 << 40) || (size_t)q.B * q.Hq * q.N * q.d > ((size_t)1 << 40))
     return fail(GBS_ERR_INVALID_ARG, "problem too large");
+  // token rows are TMA coordinates and grid indices: signed 32-bit
+  if ((size_t)q.B * q.Hq * q.N > (size_t)INT32_MAX)
+    return fail(GBS_ERR_INVALID_ARG, "problem too large: B * Hq * N must be below 2^31");
   Problem& p = *out;
   p.B = q.B; p.Hq = q.Hq; p.Hkv = q.Hkv; p.N = q.N; p.d = q.d; p.bs = q.block;
   p.Nb = (int)Nb; p.G = q.Hq / q.Hkv; p.topk = uses_topk ? q.topk : 0;

@@ -45,7 +45,9 @@
  *     q-head h reads kv-head h / (Hq / Hkv).
  *   - Supported: d in {64, 128}; block == 64; N % 64 == 0 (training/prefill);
  *     Hq % Hkv == 0; 0 <= topk <= GBS_MAX_TOPK; dtype bf16 (tensor-core path)
- *     or fp32 (exact SIMT path). S must be finite.
+ *     or fp32 (exact SIMT path). S must be finite. B * Hq * N < 2^31 (token
+ *     rows are 32-bit TMA coordinates); larger problems return
+ *     GBS_ERR_INVALID_ARG.
  */
 #ifndef GBS_H_
 #define GBS_H_

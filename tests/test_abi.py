@@ -63,6 +63,7 @@ def test_workspace_sizes(lib):
     (dict(mode="sparse", topk=-1), 1),
     (dict(mode="sparse", topk=10_000), 1),
     (dict(B=0), 1),
+    (dict(B=1024, Hq=64, Hkv=8, N=32768), 1),   # 2^31 token rows: beyond 32-bit coordinates
 ])
 def test_invalid_params_rejected_before_launch(lib, kw, status):
     args = dict(B=1, Hq=4, Hkv=2, N=256, d=64, block=64, topk=0, mode="train")
