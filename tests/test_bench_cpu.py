@@ -39,3 +39,31 @@ def test_traffic_is_tied_to_the_measured_source(tmp_path, monkeypatch):
     assert bench.traffic_for("missing") is None
     src.write_text("// kernel v2\n")  # the kernel changed since the counters were taken
     assert bench.traffic_for("k") is None
+
+
+def _union_tiling_fraction(S, k):
+    """Attended pairs / pairs the sparse forward's stages compute, for the
+    tiling that pairs query blocks 2t and 2t+1 over the union of their kept
+    blocks plus both current blocks, padded to an even count of 64-key slots,
+    two slots per 128 x 128 stage."""
+    Hq, Nb = S.shape[1], S.shape[2]
+    attended = computed = 0.0
+    for h in range(Hq):
+        kept = [set(oracle.attended_blocks(S[0, h, r], r, oracle.SPARSE, k).tolist()) for r in range(Nb)]
+        for t in range(Nb // 2):
+            r0, r1 = 2 * t, 2 * t + 1
+            slots = len(kept[r0] | kept[r1] | {r0, r1})
+            computed += (slots + (slots & 1)) * 64 * 128
+            attended += (len(kept[r0]) + len(kept[r1])) * 64 * 64 + 2 * (64 * 65 // 2)
+    return attended / computed
+
+
+def test_sparse_prefill_tiling_ceiling():
+    """On the planted N = 65536 recipe (two heads drawn), the two-query-block
+    tiles compute about twice the attended pairs: the tiling's ceiling is about
+    half the tensor peak at K = 8 and about 60% at K = 32."""
+    from gated_block_sparse_gate_b200.inputs import WORKLOADS, make_prefill_inputs
+    w = WORKLOADS["sparse_prefill_bf16_n65536"]
+    S = make_prefill_inputs(w, Hq=2, Hkv=1, with_grad=False)["S"].numpy().astype(np.float64)
+    f8, f32 = _union_tiling_fraction(S, 8), _union_tiling_fraction(S, 32)
+    assert 0.45 < f8 < 0.56 and 0.55 < f32 < 0.65, (f8, f32)
