@@ -11,8 +11,10 @@
 // The work is bound by HBM: every selected block streams 64 keys and 64 values
 // once. Split kernel: grid (B*Hq, splits); each CTA takes a contiguous share of
 // the (selected + current) block list; a group of D/8 lanes owns one key row
-// and loads it with 16-byte vector loads (eight loads in flight per lane before
-// any arithmetic), reduces the dot product with shuffles and keeps an online
+// and loads it with 16-byte vector loads (for bf16 the block's eight key and
+// eight value rows of a lane are all in flight before any arithmetic; fp32
+// loads the values after the scores), reduces the dot product with shuffles
+// and keeps an online
 // softmax state. The CTA merges its eight groups and writes one partial
 // (m, l, acc[D]) per split; the combine kernel merges the splits.
 //
@@ -63,6 +65,13 @@ __device__ __forceinline__ Vec8 load8<float>(const float* ptr) {
   return r;
 }
 
+// Element i of eight bf16 values held as one 16-byte word (element 0 in the
+// low half of .x); a bf16 widens to fp32 by a 16-bit shift.
+__device__ __forceinline__ float bf16_elem(const uint4& u, int i) {
+  const uint32_t w = i < 2 ? u.x : (i < 4 ? u.y : (i < 6 ? u.z : u.w));
+  return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));
+}
+
 // Online-softmax state of one lane group (log2 domain).
 struct State {
   float m, l, acc[8];
@@ -82,6 +91,7 @@ decode_split_kernel(Problem p, const T* __restrict__ q, const T* __restrict__ Kc
   constexpr int GPW = 32 / LPK;          // key groups per warp
   constexpr int NGROUPS = (kThreads / 32) * GPW;
   constexpr int ROWS_PER_GROUP = kBS / NGROUPS;
+  constexpr bool kRaw = sizeof(T) == 2;
   __shared__ float s_m[NGROUPS][NH], s_l[NGROUPS][NH];
   __shared__ float s_acc[NGROUPS][NH][D];
   __shared__ int s_row0[kEntChunk];  // first cache row (units of D elements); -1: skip it
@@ -161,8 +171,56 @@ decode_split_kernel(Problem p, const T* __restrict__ q, const T* __restrict__ Kc
     const int nrows = s_rows[e - cs];
     // rows handled by this group inside the block
     const int row0 = group * ROWS_PER_GROUP;
-    Vec8 kvr[ROWS_PER_GROUP];
     float s[NH][ROWS_PER_GROUP];
+    if constexpr (kRaw) {
+      // bf16: the block's key and value rows are all requested before any
+      // arithmetic (one memory latency per block), and held as raw 16-byte
+      // words, which costs the registers that eight converted rows would
+      uint4 kr[ROWS_PER_GROUP], vr[ROWS_PER_GROUP];
+#pragma unroll
+      for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) {
+        const int row = min(row0 + rr, nrows - 1);
+        kr[rr] = __ldg(reinterpret_cast<const uint4*>(Kc + base + (size_t)row * D + sub * 8));
+      }
+#pragma unroll
+      for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) {
+        const int row = min(row0 + rr, nrows - 1);
+        vr[rr] = __ldg(reinterpret_cast<const uint4*>(Vc + base + (size_t)row * D + sub * 8));
+      }
+#pragma unroll
+      for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) {
+#pragma unroll
+        for (int g = 0; g < NH; ++g) {
+          float d = 0.f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) d = fmaf(qv[g].v[i], bf16_elem(kr[rr], i), d);
+#pragma unroll
+          for (int o = LPK / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+          s[g][rr] = (row0 + rr < nrows) ? d + bias2 : -INFINITY;
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < NH; ++g) {
+        float mloc = st[g].m;
+#pragma unroll
+        for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) mloc = fmaxf(mloc, s[g][rr]);
+        if (mloc > -INFINITY) {
+          const float corr = exp2f(st[g].m - mloc);
+          st[g].l *= corr;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) st[g].acc[i] *= corr;
+          st[g].m = mloc;
+#pragma unroll
+          for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) {
+            const float pr = exp2f(s[g][rr] - mloc);
+            st[g].l += pr;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) st[g].acc[i] = fmaf(pr, bf16_elem(vr[rr], i), st[g].acc[i]);
+          }
+        }
+      }
+    } else {
+    Vec8 kvr[ROWS_PER_GROUP];
 #pragma unroll
     for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) {
       const int row = min(row0 + rr, nrows - 1);
@@ -204,6 +262,7 @@ decode_split_kernel(Problem p, const T* __restrict__ q, const T* __restrict__ Kc
           for (int i = 0; i < 8; ++i) st[g].acc[i] = fmaf(pr, kvr[rr].v[i], st[g].acc[i]);
         }
       }
+    }
     }
   }
   }
