@@ -386,14 +386,18 @@ gbs_status gbs_decode_ex(const gbs_params* in, const gbs_kv_layout* kvl, const v
   const int cta_rows = grouped ? p.B * p.Hkv * (p.G / decode_heads_per_cta(p, true)) : p.B * p.Hq;
   int splits = num_splits;
   if (splits == 0) {
-    // enough CTAs for about four waves of the split kernel's resident CTAs
-    // (measured best on the 64 x 131072 decode: 3 splits per q-head row, 2 per
-    // shared-selection row)
+    // Shares of at most 17 blocks per CTA, and at least two waves of the split
+    // kernel's resident CTAs. On the 64 x 131072, K = 32 decode both variants
+    // are fastest at 2 splits (16-17 blocks a CTA): per q-head row 0.363 ms
+    // against 0.375 / 0.373 ms at 1 / 3; per shared-selection row 0.175 ms
+    // against 0.179 ms at 3 and 0.187 ms at 6.
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int waves_ctas = 4 * sms * decode_resident_ctas(p, grouped);
-    splits = (waves_ctas + cta_rows - 1) / cta_rows;
+    const int two_waves = 2 * sms * decode_resident_ctas(p, grouped);
+    const int by_share = (n_ent + 16) / 17;
+    const int by_waves = (two_waves + cta_rows - 1) / cta_rows;
+    splits = by_share > by_waves ? by_share : by_waves;
   }
   if (splits > n_ent) splits = n_ent;
   if (splits > kMaxSplits) splits = kMaxSplits;

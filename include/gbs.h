@@ -172,7 +172,9 @@ GBS_API gbs_status gbs_bwd(const gbs_params* p, const void* Q, const void* K, co
  *   p->mode GBS_THRESHOLD keeps only those of them whose gate reaches p->tau
  *   (as in gbs_fwd); any other mode value selects plain Top-K.
  *   O [B,Hq,d] out (p->dtype); LSE [B,Hq] fp32 out.
- *   num_splits: partitions of the selected blocks per (b, h); 0 = automatic.
+ *   num_splits: partitions of the selected blocks per (b, h); 0 = automatic
+ *               (at most 17 blocks per partition, and at least two waves of
+ *               resident CTAs).
  *   ws: gbs_workspace_bytes(p, GBS_OP_DECODE) bytes. */
 GBS_API gbs_status gbs_decode(const gbs_params* p, const void* q, const void* Kc, const void* Vc,
                       const float* S, void* O, float* LSE, int num_splits, void* ws,
