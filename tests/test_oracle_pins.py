@@ -54,33 +54,6 @@ def test_single_block_is_dense_causal():
     assert np.all(dS == 0.0)
 
 
-def test_closed_form_three_tokens():
-    """Hand-derived case, block = 1 (per-token units), d = 1, q = 0.
-
-    Row 2 has history {0, 1} with scores (ln 3, 0): gates (3/4, 1/4); the
-    current token has bias 0; all q.k are 0. Softmax weights are therefore
-    (3/8, 1/8, 1/2); with v = (1, 2, 3) the output is 17/8 and LSE = ln 2.
-    With dO = 1 on row 2: dZ = P (v - O) = (-27/64, -1/64, 28/64), so
-    G = (-27/64, -1/64) and dS = G - g * sum(G) = (-3/32, +3/32).
-    Row 1 has a single historical token: gate 1, weights (1/2, 1/2).
-    """
-    Q = np.zeros((1, 1, 3, 1))
-    K = np.array([1.0, -2.0, 0.5]).reshape(1, 1, 3, 1)
-    V = np.array([1.0, 2.0, 3.0]).reshape(1, 1, 3, 1)
-    S = np.zeros((1, 1, 3, 3))
-    S[0, 0, 2, 0] = math.log(3.0)
-    S[0, 0, 1, 0] = 5.0
-    O, LSE = oracle.gated_attention_forward(Q, K, V, S, 1)
-    assert np.allclose(O[0, 0, :, 0], [1.0, 1.5, 17.0 / 8.0], rtol=0, atol=1e-14)
-    assert np.allclose(LSE[0, 0], [0.0, math.log(2.0), math.log(2.0)], rtol=0, atol=1e-14)
-    dO = np.zeros((1, 1, 3, 1))
-    dO[0, 0, 2, 0] = 1.0
-    dQ, dK, dV, dS, Gs = oracle.gated_attention_backward(Q, K, V, S, dO, 1)
-    assert np.allclose(Gs[0, 0, 2, :2], [-27 / 64, -1 / 64], atol=1e-14)
-    assert np.allclose(dS[0, 0, 2, :2], [-3 / 32, 3 / 32], atol=1e-14)
-    assert np.allclose(dV[0, 0, :, 0], [3 / 8, 1 / 8, 1 / 2], atol=1e-14)
-
-
 def test_constant_scores_give_uniform_gates():
     """A constant score row gives g = 1/|A|, i.e. log-gate -ln r (train) or -ln K."""
     S = np.full((1, 1, 9, 9), 0.7)
