@@ -98,6 +98,95 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+# Device types whose memory the kernels may be given; only the unit tests of
+# the checks below widen it (to "meta", which has shapes but no storage).
+_DEVICE_TYPES = ("cuda",)
+_F32 = (torch.float32,)
+_I32 = (torch.int32,)
+_U8 = (torch.uint8,)
+
+
+def _invalid(where, detail):
+    return GbsError(1, where, detail)
+
+
+def _device(where, name, t):
+    """The device of the call's anchor tensor, which must be a CUDA tensor."""
+    if not isinstance(t, torch.Tensor):
+        raise _invalid(where, f"{name} must be a torch.Tensor")
+    if t.device.type not in _DEVICE_TYPES:
+        raise _invalid(where, f"{name} is on {t.device}; the kernels need CUDA memory")
+    return t.device
+
+
+def _need(where, name, t, shape, dtypes, device):
+    """t is a contiguous tensor on ``device`` with one of ``dtypes`` and, unless
+    ``shape`` is None, exactly that shape: the layout the C ABI reads."""
+    if not isinstance(t, torch.Tensor):
+        raise _invalid(where, f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise _invalid(where, f"{name} is on {t.device}; expected {device}")
+    if t.dtype not in dtypes:
+        raise _invalid(where, f"{name} has dtype {t.dtype}; expected {' or '.join(map(str, dtypes))}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise _invalid(where, f"{name} has shape {tuple(t.shape)}; expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise _invalid(where, f"{name} must be contiguous")
+
+
+def _act_dtype(where, name, t):
+    if t.dtype not in DTYPES:
+        raise _invalid(where, f"{name} has dtype {t.dtype}; expected torch.bfloat16 or torch.float32")
+    return (t.dtype,)
+
+
+def _check_prefill(where, Q, K, V, S, block, outs=()):
+    """Q [B,Hq,N,d], K and V [B,Hkv,N,d] of Q's dtype, S [B,Hq,Nb,Nb] fp32, and
+    each (name, tensor, shape, dtypes) of ``outs``; returns (device, shape dict)."""
+    dev = _device(where, "Q", Q)
+    if Q.dim() != 4 or not isinstance(K, torch.Tensor) or K.dim() != 4:
+        raise _invalid(where, "Q and K must be 4-D: [B, H, N, d]")
+    B, Hq, N, d = Q.shape
+    Hkv = K.shape[1]
+    Nb = -(-N // block)
+    act = _act_dtype(where, "Q", Q)
+    _need(where, "Q", Q, (B, Hq, N, d), act, dev)
+    _need(where, "K", K, (B, Hkv, N, d), act, dev)
+    _need(where, "V", V, (B, Hkv, N, d), act, dev)
+    _need(where, "S", S, (B, Hq, Nb, Nb), _F32, dev)
+    for name, t, shape, dtypes in outs:
+        _need(where, name, t, shape, dtypes, dev)
+    return dev
+
+
+def _check_decode(where, q, Kc, Vc, S, L, block, block_table=None, seq_lens=None,
+                  group_shared=False, outs=()):
+    """q [B,Hq,d]; a cache [B,Hkv,L,d] or, with a block table, page pools
+    [pages,Hkv,block,d]; S [B,Hq,Nb] (group-shared: [B,Hkv,Nb]) fp32; an int32
+    block table [B, max_blocks] and int32 lengths [B]."""
+    dev = _device(where, "q", q)
+    if q.dim() != 3 or not isinstance(Kc, torch.Tensor) or Kc.dim() != 4:
+        raise _invalid(where, "q must be [B, Hq, d] and the cache 4-D")
+    B, Hq, d = q.shape
+    Hkv = Kc.shape[1]
+    Nb = -(-L // block)
+    act = _act_dtype(where, "q", q)
+    _need(where, "q", q, (B, Hq, d), act, dev)
+    cache = (Kc.shape[0], Hkv, block, d) if block_table is not None else (B, Hkv, L, d)
+    _need(where, "Kc", Kc, cache, act, dev)
+    _need(where, "Vc", Vc, cache, act, dev)
+    _need(where, "S", S, (B, Hkv if group_shared else Hq, Nb), _F32, dev)
+    if block_table is not None:
+        _need(where, "block_table", block_table, None, _I32, dev)
+        if block_table.dim() != 2 or block_table.shape[0] != B:
+            raise _invalid(where, f"block_table must be [B={B}, max_blocks]")
+    if seq_lens is not None:
+        _need(where, "seq_lens", seq_lens, (B,), _I32, dev)
+    for name, t, shape, dtypes in outs:
+        _need(where, name, t, shape, dtypes, dev)
+    return dev
+
+
 def make_params(B, Hq, Hkv, N, d, block=64, topk=0, mode="train", dtype=torch.bfloat16, scale=0.0,
                 tau=0.0):
     return Params(B, Hq, Hkv, N, d, block, topk, MODES[mode], DTYPES[dtype], float(scale),
@@ -125,10 +214,13 @@ def _prefill_params(Q, K, S, block, topk, mode, scale, tau=0.0):
 def select(S, block=64, topk=0, mode="sparse", N=None, tau=0.0, stream=None):
     """K1: (idx, cnt, logg, slse) for S [B, Hq, Nb, Nb]."""
     lib = load_library()
+    dev = _device("gbs_select", "S", S)
+    if S.dim() != 4:
+        raise _invalid("gbs_select", "S must be [B, Hq, Nb, Nb]")
     B, Hq, Nb, _ = S.shape
+    _need("gbs_select", "S", S, (B, Hq, Nb, Nb), _F32, dev)
     N = N if N is not None else Nb * block
     p = make_params(B, Hq, Hq, N, 64, block, topk, mode, torch.float32, tau=tau)
-    dev = S.device
     idx = cnt = logg = None
     if mode != "train":
         idx = torch.empty(B, Hq, Nb, topk, dtype=torch.int32, device=dev)
@@ -144,11 +236,15 @@ def forward(Q, K, V, S, block=64, mode="train", topk=0, scale=0.0, out=None, lse
             tau=0.0, stream=None):
     """Gated attention forward: returns (O, LSE)."""
     lib = load_library()
+    _check_prefill("gbs_fwd", Q, K, V, S, block)
     p = _prefill_params(Q, K, S, block, topk, mode, scale, tau)
     O = out if out is not None else torch.empty_like(Q)
     LSE = lse if lse is not None else torch.empty(Q.shape[:3], dtype=torch.float32, device=Q.device)
     if ws is None:
         ws = alloc_workspace(p, OP_FWD, Q.device)
+    _check_prefill("gbs_fwd", Q, K, V, S, block,
+                   outs=(("O", O, Q.shape, (Q.dtype,)), ("LSE", LSE, Q.shape[:3], _F32),
+                         ("ws", ws, None, _U8)))
     _check(lib.gbs_fwd(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(S), _ptr(O), _ptr(LSE),
                        _ptr(ws), ws.numel(), _stream(stream)), "gbs_fwd")
     return O, LSE
@@ -158,12 +254,19 @@ def backward(Q, K, V, S, O, LSE, dO, block=64, scale=0.0, grads=None, ws=None, m
              topk=0, tau=0.0, stream=None):
     """Backward of ``forward`` with the same mode/topk/tau: returns (dQ, dK, dV, dS)."""
     lib = load_library()
+    _check_prefill("gbs_bwd", Q, K, V, S, block)
     p = _prefill_params(Q, K, S, block, topk, mode, scale, tau)
     if grads is None:
         grads = (torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V), torch.empty_like(S))
     dQ, dK, dV, dS = grads
     if ws is None:
         ws = alloc_workspace(p, OP_BWD, Q.device)
+    act = (Q.dtype,)
+    _check_prefill("gbs_bwd", Q, K, V, S, block,
+                   outs=(("O", O, Q.shape, act), ("LSE", LSE, Q.shape[:3], _F32),
+                         ("dO", dO, Q.shape, act), ("dQ", dQ, Q.shape, act),
+                         ("dK", dK, K.shape, act), ("dV", dV, V.shape, act),
+                         ("dS", dS, S.shape, _F32), ("ws", ws, None, _U8)))
     _check(lib.gbs_bwd(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(S), _ptr(O), _ptr(LSE),
                        _ptr(dO), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dS), _ptr(ws), ws.numel(),
                        _stream(stream)), "gbs_bwd")
@@ -177,8 +280,9 @@ def decode(q, Kc, Vc, S, L=None, block=64, topk=32, scale=0.0, num_splits=0, out
     ``tau`` set selects threshold mode (blocks whose gate reaches tau, at most topk).
     """
     lib = load_library()
-    B, Hq, d = q.shape
     L = Kc.shape[2] if L is None else L
+    _check_decode("gbs_decode", q, Kc, Vc, S, L, block)
+    B, Hq, d = q.shape
     mode = "sparse" if tau is None else "threshold"
     p = make_params(B, Hq, Kc.shape[1], L, d, block, topk, mode, q.dtype, scale,
                     0.0 if tau is None else tau)
@@ -186,6 +290,9 @@ def decode(q, Kc, Vc, S, L=None, block=64, topk=32, scale=0.0, num_splits=0, out
     LSE = lse if lse is not None else torch.empty(B, Hq, dtype=torch.float32, device=q.device)
     if ws is None:
         ws = alloc_workspace(p, OP_DECODE, q.device)
+    _check_decode("gbs_decode", q, Kc, Vc, S, L, block,
+                  outs=(("O", O, q.shape, (q.dtype,)), ("LSE", LSE, (B, Hq), _F32),
+                        ("ws", ws, None, _U8)))
     _check(lib.gbs_decode(ctypes.byref(p), _ptr(q), _ptr(Kc), _ptr(Vc), _ptr(S), _ptr(O), _ptr(LSE),
                           num_splits, _ptr(ws), ws.numel(), _stream(stream)), "gbs_decode")
     return O, LSE
@@ -200,6 +307,7 @@ def decode_ex(q, Kc, Vc, S, L, block=64, topk=32, scale=0.0, num_splits=0, block
     [num_pages, Hkv, block, d]; ``seq_lens`` (int32 [B]) gives each length;
     with ``group_shared`` S is [B, Hkv, Nb]. Returns (O, LSE)."""
     lib = load_library()
+    _check_decode("gbs_decode_ex", q, Kc, Vc, S, L, block, block_table, seq_lens, group_shared)
     B, Hq, d = q.shape
     mode = "sparse" if tau is None else "threshold"
     p = make_params(B, Hq, Kc.shape[1], L, d, block, topk, mode, q.dtype, scale,
@@ -212,6 +320,9 @@ def decode_ex(q, Kc, Vc, S, L, block=64, topk=32, scale=0.0, num_splits=0, block
     LSE = lse if lse is not None else torch.empty(B, Hq, dtype=torch.float32, device=q.device)
     if ws is None:
         ws = alloc_workspace(p, OP_DECODE, q.device)
+    _check_decode("gbs_decode_ex", q, Kc, Vc, S, L, block, block_table, seq_lens, group_shared,
+                  outs=(("O", O, q.shape, (q.dtype,)), ("LSE", LSE, (B, Hq), _F32),
+                        ("ws", ws, None, _U8)))
     _check(lib.gbs_decode_ex(ctypes.byref(p), ctypes.byref(kv), _ptr(q), _ptr(Kc), _ptr(Vc), _ptr(S),
                              _ptr(O), _ptr(LSE), num_splits, _ptr(ws), ws.numel(), _stream(stream)),
            "gbs_decode_ex")
@@ -236,6 +347,7 @@ def launch_count() -> int:
 
 def check(ws, stream=None):
     """Raises GbsError if a kernel recorded a device-side error in ``ws``."""
+    _device("gbs_check", "ws", ws)
     _check(load_library().gbs_check(_ptr(ws), _stream(stream)), "gbs_check")
 
 
@@ -251,13 +363,16 @@ def decode_noalloc(q, Kc, Vc, S, L=None, block=64, topk=32, scale=0.0, num_split
     vp = ctypes.c_void_p
     f.restype = ctypes.c_int
     f.argtypes = [ctypes.POINTER(Params), vp, vp, vp, vp, vp, vp, ctypes.c_int, vp]
-    B, Hq, d = q.shape
     L = Kc.shape[2] if L is None else L
+    _check_decode("gbs_decode_noalloc", q, Kc, Vc, S, L, block)
+    B, Hq, d = q.shape
     mode = "sparse" if tau is None else "threshold"
     p = make_params(B, Hq, Kc.shape[1], L, d, block, topk, mode, q.dtype, scale,
                     0.0 if tau is None else tau)
     O = out if out is not None else torch.empty_like(q)
     LSE = lse if lse is not None else torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    _check_decode("gbs_decode_noalloc", q, Kc, Vc, S, L, block,
+                  outs=(("O", O, q.shape, (q.dtype,)), ("LSE", LSE, (B, Hq), _F32)))
     _check(f(ctypes.byref(p), _ptr(q), _ptr(Kc), _ptr(Vc), _ptr(S), _ptr(O), _ptr(LSE), num_splits,
              _stream(stream)), "gbs_decode_noalloc")
     return O, LSE
