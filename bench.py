@@ -488,8 +488,9 @@ def bench_decode(dev, peaks, reps=10):
     return out
 
 
-def cpu_baseline_sample(w, budget_s=30.0):
-    """The float64 oracle on kv-group 0 (4 of 32 q-heads) of the training workload."""
+def cpu_baseline_sample(w, min_s=10.0):
+    """The float64 oracle on whole kv groups (G q-heads each) of the training
+    workload, group after group until at least ``min_s`` seconds are timed."""
     import numpy as np
 
     import oracle
@@ -497,13 +498,18 @@ def cpu_baseline_sample(w, budget_s=30.0):
     x = make_prefill_inputs(w)
     G = w.Hq // w.Hkv
     f64 = lambda t: t.float().numpy().astype(np.float64)  # noqa: E731
-    Q, K, V, dO = f64(x["Q"][:, :G]), f64(x["K"][:, :1]), f64(x["V"][:, :1]), f64(x["dO"][:, :G])
-    S = x["S"][:, :G].numpy()
-    t0 = time.perf_counter()
-    oracle.gated_attention_forward(Q, K, V, S, w.block)
-    oracle.gated_attention_backward(Q, K, V, S, dO, w.block)
-    dt = time.perf_counter() - t0
-    fl = 14.0 * w.d * train_pairs_per_head(w.Nb, w.block) * G
+    dt, groups = 0.0, 0
+    while groups < w.Hkv and dt < min_s:
+        hs = slice(groups * G, (groups + 1) * G)
+        kv = slice(groups, groups + 1)
+        Q, K, V, dO = f64(x["Q"][:, hs]), f64(x["K"][:, kv]), f64(x["V"][:, kv]), f64(x["dO"][:, hs])
+        S = x["S"][:, hs].numpy()
+        t0 = time.perf_counter()
+        oracle.gated_attention_forward(Q, K, V, S, w.block)
+        oracle.gated_attention_backward(Q, K, V, S, dO, w.block)
+        dt += time.perf_counter() - t0
+        groups += 1
+    fl = 14.0 * w.d * train_pairs_per_head(w.Nb, w.block) * G * groups
     threads = os.cpu_count()
     try:
         from threadpoolctl import threadpool_info
@@ -511,8 +517,10 @@ def cpu_baseline_sample(w, budget_s=30.0):
     except Exception:  # noqa: BLE001
         pass
     return {"value": fl / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"float64 NumPy oracle, forward+backward of kv-group 0 (4 of 32 q-heads) of "
-                      f"{w.name}; {dt:.1f} s; host cores {os.cpu_count()}"}
+            "sample": f"float64 NumPy oracle, forward+backward of "
+                      f"{'kv group 0' if groups == 1 else f'kv groups 0-{groups - 1}'} "
+                      f"({groups * G} of {w.Hq} q-heads) of {w.name}; {dt:.1f} s; "
+                      f"host cores {os.cpu_count()}"}
 
 
 # -------------------------------------------------------------- reference arm
