@@ -357,6 +357,9 @@ gbs_status gbs_decode_ex(const gbs_params* in, const gbs_kv_layout* kvl, const v
         return fail(GBS_ERR_INVALID_ARG, "max_blocks (%d) is below ceil(N / block) = %d",
                     kvl->max_blocks, p.Nb);
       if (kvl->num_pages <= 0) return fail(GBS_ERR_INVALID_ARG, "num_pages must be positive");
+      // a page's first cache row is a signed 32-bit index
+      if ((size_t)kvl->num_pages * p.Hkv * p.bs > (size_t)INT32_MAX)
+        return fail(GBS_ERR_INVALID_ARG, "num_pages * Hkv * block must be below 2^31");
       if ((uintptr_t)kvl->block_table & 3u)
         return fail(GBS_ERR_INVALID_ARG, "block_table is not 4-byte aligned");
     }

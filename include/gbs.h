@@ -190,7 +190,8 @@ GBS_API gbs_status gbs_decode(const gbs_params* p, const void* q, const void* Kc
  *                block of every kv head per page). Only the first
  *                ceil(L_b / block) entries of a row are read.
  *   max_blocks   row stride of block_table, >= ceil(p->N / block).
- *   num_pages    pages in each pool; an entry outside [0, num_pages) is
+ *   num_pages    pages in each pool, with num_pages * Hkv * block < 2^31;
+ *                an entry outside [0, num_pages) is
  *                skipped on the device and reported by gbs_check as
  *                GBS_ERR_INVALID_ARG (that sequence's output is then wrong).
  *   seq_lens     NULL: every sequence has length L = p->N. Else a DEVICE array

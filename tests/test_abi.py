@@ -141,7 +141,8 @@ def test_binding_fails_loudly_without_library(tmp_path):
         gb._lib = saved
 
 
-@pytest.mark.parametrize("field,value", [("max_blocks", 3), ("num_pages", 0), ("group_shared", 2)])
+@pytest.mark.parametrize("field,value", [("max_blocks", 3), ("num_pages", 0), ("group_shared", 2),
+                                         ("num_pages", 1 << 25)])  # 2^25 pages x 2 heads x 64 rows
 def test_decode_ex_layout_checks(lib, field, value):
     """Paged-layout fields are checked before any launch."""
     p = gb.make_params(2, 8, 2, 1000, 64, 64, 4, "sparse")  # Nb = 16
