@@ -67,3 +67,36 @@ def test_sparse_prefill_tiling_ceiling():
     S = make_prefill_inputs(w, Hq=2, Hkv=1, with_grad=False)["S"].numpy().astype(np.float64)
     f8, f32 = _union_tiling_fraction(S, 8), _union_tiling_fraction(S, 32)
     assert 0.45 < f8 < 0.56 and 0.55 < f32 < 0.65, (f8, f32)
+
+
+def _backward_tiling_fraction(S, k, G):
+    """Attended pairs / pairs the sparse backward's steps compute: per 128-key
+    tile (blocks 2u, 2u+1) of a kv group, every (q-head, query block) that keeps
+    either block (or is one of them) is an entry, two entries per 128 x 128 step."""
+    Nb = S.shape[2]
+    kept = [[set(oracle.attended_blocks(S[0, h, r], r, oracle.SPARSE, k).tolist()) | {r}
+             for r in range(Nb)] for h in range(G)]
+    attended = computed = 0.0
+    for u in range(Nb // 2):
+        tile = {2 * u, 2 * u + 1}
+        entries = 0
+        for h in range(G):
+            for r in range(2 * u, Nb):
+                n = len(kept[h][r] & tile)
+                if n:
+                    entries += 1
+                    diag = r in tile
+                    attended += (n - diag) * 64 * 64 + diag * (64 * 65 // 2)
+        computed += ((entries + 1) // 2) * 128 * 128
+    return attended / computed
+
+
+def test_sparse_backward_tiling_ceiling():
+    """On one kv group of the planted N = 65536 recipe the backward's steps
+    compute about twice the attended pairs: its ceiling is about half the
+    tensor peak."""
+    from gated_block_sparse_gate_b200.inputs import WORKLOADS, make_prefill_inputs
+    w = WORKLOADS["sparse_prefill_bf16_n65536"]
+    S = make_prefill_inputs(w, Hq=4, Hkv=1, with_grad=False)["S"].numpy().astype(np.float64)
+    f8, f32 = _backward_tiling_fraction(S, 8, 4), _backward_tiling_fraction(S, 32, 4)
+    assert 0.43 < f8 < 0.52 and 0.48 < f32 < 0.57, (f8, f32)
