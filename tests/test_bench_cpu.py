@@ -100,3 +100,17 @@ def test_sparse_backward_tiling_ceiling():
     S = make_prefill_inputs(w, Hq=4, Hkv=1, with_grad=False)["S"].numpy().astype(np.float64)
     f8, f32 = _backward_tiling_fraction(S, 8, 4), _backward_tiling_fraction(S, 32, 4)
     assert 0.43 < f8 < 0.52 and 0.48 < f32 < 0.57, (f8, f32)
+
+
+def test_reference_arm_prints_the_contract_line(capsys):
+    """bench.py --impl reference: the oracle on the host cores, one JSON line."""
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "1"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0 and line["steps"] == 1
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["unit"] == line["unit"]
+    assert line["config"]["workload"] == "train_bf16_n8192"
