@@ -135,7 +135,12 @@ GBS_API gbs_status gbs_check(const void* ws, void* stream);
 GBS_API gbs_status gbs_select(const gbs_params* p, const float* S, int32_t* idx, int32_t* cnt,
                       float* logg, float* slse, void* stream);
 
-/* Gated attention forward (select + attention).
+/* Gated attention forward (select + attention): softmax attention whose
+ * logits carry the log gates of the attended historical blocks and 0 for the
+ * current block (blog section "The Logit Injection Mechanism"; poster and HF
+ * page Abstracts for the training and Top-K modes; blog section
+ * "Implementation and Efficiency" for the threshold mode and the blockwise
+ * processing that never forms the N x N matrix).
  *   Q [B,Hq,N,d], K/V [B,Hkv,N,d] in p->dtype; S [B,Hq,Nb,Nb] fp32.
  *   O [B,Hq,N,d] out (p->dtype); LSE [B,Hq,N] fp32 out, natural log of
  *   sum_j exp z_ij with z including scale and bias.
@@ -164,7 +169,10 @@ GBS_API gbs_status gbs_bwd(const gbs_params* p, const void* Q, const void* K, co
                    void* dQ, void* dK, void* dV, float* dS, void* ws, size_t ws_bytes,
                    void* stream);
 
-/* Sparse decode: one query per sequence at position L-1 (L = p->N).
+/* Sparse decode: one query per sequence at position L-1 (L = p->N), the
+ * inference-time use of the method with a fixed budget of context blocks per
+ * query (poster Abstract) and the current block always retained (HF page
+ * Abstract).
  *   q [B,Hq,d]; Kc/Vc [B,Hkv,L,d] (p->dtype); S [B,Hq,Nb] fp32 with
  *   Nb = ceil(L / block): scores of the current block's row over key blocks
  *   c < cur = (L-1)/block. Attends the Top-K (p->topk) historical blocks with
