@@ -5,7 +5,6 @@ import os
 import re
 
 import pytest
-import torch
 
 from gated_block_sparse_gate_b200 import binding as gb
 from gated_block_sparse_gate_b200.build import build
