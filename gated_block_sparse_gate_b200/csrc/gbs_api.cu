@@ -222,7 +222,7 @@ const char* gbs_status_string(gbs_status s) {
 const char* gbs_last_error(void) { return g_last_error; }
 
 size_t gbs_workspace_bytes(const gbs_params* in, int op) {
-  Problem p;
+  Problem p{};
   if (resolve(in, op, &p) != GBS_OK) return 0;
   if (op == GBS_OP_FWD) return carve_fwd(p, nullptr).bytes;
   if (op == GBS_OP_BWD) return carve_bwd(p, nullptr).bytes;
@@ -248,7 +248,7 @@ gbs_status gbs_check(const void* ws, void* stream) {
 gbs_status gbs_select(const gbs_params* in, const float* S, int32_t* idx, int32_t* cnt,
                       float* logg, float* slse, void* stream) {
   g_last_error[0] = 0;
-  Problem p;
+  Problem p{};
   gbs_status s = resolve(in, GBS_OP_FWD, &p);
   if (s != GBS_OK) return s;
   const bool sparse = p.mode != GBS_TRAIN;
@@ -265,7 +265,7 @@ gbs_status gbs_select(const gbs_params* in, const float* S, int32_t* idx, int32_
 gbs_status gbs_fwd(const gbs_params* in, const void* Q, const void* K, const void* V,
                    const float* S, void* O, float* LSE, void* ws, size_t ws_bytes, void* stream) {
   g_last_error[0] = 0;
-  Problem p;
+  Problem p{};
   gbs_status s = resolve(in, GBS_OP_FWD, &p);
   if (s != GBS_OK) return s;
   const void* ptrs[] = {Q, K, V, S, O, LSE};
@@ -298,7 +298,7 @@ gbs_status gbs_bwd(const gbs_params* in, const void* Q, const void* K, const voi
                    const float* S, const void* O, const float* LSE, const void* dO, void* dQ,
                    void* dK, void* dV, float* dS, void* ws, size_t ws_bytes, void* stream) {
   g_last_error[0] = 0;
-  Problem p;
+  Problem p{};
   gbs_status s = resolve(in, GBS_OP_BWD, &p);
   if (s != GBS_OK) return s;
   const void* ptrs[] = {Q, K, V, S, O, LSE, dO, dQ, dK, dV, dS};
@@ -339,7 +339,7 @@ gbs_status gbs_decode_ex(const gbs_params* in, const gbs_kv_layout* kvl, const v
                          const void* Kc, const void* Vc, const float* S, void* O, float* LSE,
                          int num_splits, void* ws, size_t ws_bytes, void* stream) {
   g_last_error[0] = 0;
-  Problem p;
+  Problem p{};
   gbs_status s = resolve(in, GBS_OP_DECODE, &p);
   if (s != GBS_OK) return s;
   const void* ptrs[] = {q, Kc, Vc, S, O, LSE};
