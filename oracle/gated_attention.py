@@ -49,7 +49,8 @@ over all of H_r) in sparse mode.
 
 Parity pins (see tests/test_oracle_pins.py): dense causal attention through
 torch's SDPA; SDPA with an additive mask plus autograd for every gradient
-including dS; central finite differences; gate rows summing to one; dS rows
+including dS; the training normaliser slse against torch's masked log_softmax
+and a constant-row closed form; central finite differences; gate rows summing to one; dS rows
 summing to zero; shift invariance in S; Top-K against a brute-force rank count;
 full-budget Top-K equal to training mode; a hand-derived closed form; decode
 equal to the last row of sparse prefill; GQA equal to repeated KV heads; paged

@@ -171,6 +171,35 @@ def test_gate_rows_sum_to_one():
                     assert abs(np.exp(logg[b, h, r, :n]).sum() - 1.0) < 1e-14
 
 
+def _slse_pin_error(select):
+    """Largest deviation of select_blocks' slse from the log-normaliser of the
+    training gates as torch.log_softmax computes it over each row's history
+    c < r (HF page Abstract: gates normalised over the historical blocks), plus
+    the closed form of a constant row (slse = a + ln r) and -inf at r = 0."""
+    import torch
+
+    S = np.random.default_rng(3).standard_normal((2, 3, 11, 11)) * math.sqrt(2)
+    slse = select(S, 11, None, mode=oracle.TRAIN)[3]
+    err = 0.0
+    hist = torch.arange(11)[None, :] < torch.arange(11)[:, None]
+    ls = torch.log_softmax(torch.as_tensor(S).masked_fill(~hist, -math.inf), dim=-1).numpy()
+    for b in range(2):
+        for h in range(3):
+            if slse[b, h, 0] != -np.inf:
+                return math.inf
+            for r in range(1, 11):
+                err = max(err, float(np.max(np.abs((S[b, h, r, :r] - slse[b, h, r]) - ls[b, h, r, :r]))))
+    a = 0.7
+    const = select(np.full((1, 1, 9, 9), a), 9, None, mode=oracle.TRAIN)[3]
+    for r in range(1, 9):
+        err = max(err, abs(const[0, 0, r] - (a + math.log(r))))
+    return err
+
+
+def test_select_slse_is_history_normaliser():
+    assert _slse_pin_error(oracle.select_blocks) < 1e-12
+
+
 def test_dS_rows_sum_to_zero_and_G_rows_cancel():
     Q, K, V, S, dO = _rand(8, 1, 2, 2, 80, 8, 16)
     for kw in ({}, dict(mode=oracle.SPARSE, topk=2)):
@@ -428,3 +457,9 @@ def test_pins_catch_current_block_in_history():
     O, _ = m.gated_attention_forward(Q, K, V, S, 16, gate="ones")
     O_ref, _ = sdpa_dense_causal(Q, K, V)
     assert rel_err(O, O_ref) > 1e-3
+
+
+def test_pins_catch_slse_over_current_block():
+    m = _mutant("slse[b, h, r] = _logsumexp(_as_f64(S[b, h, r, :r]))",
+                "slse[b, h, r] = _logsumexp(_as_f64(S[b, h, r, :r + 1]))")
+    assert _slse_pin_error(m.select_blocks) > 1e-3
