@@ -2,10 +2,12 @@
 """Benchmark of the gated block-sparse attention hot path on B200.
 
 Headline: one training step of the hot path (gate normalisation, gated
-forward, gated backward with dS) on the training workload
-B=1, Hq=32, Hkv=8, d=128, N=8192, block 64, bf16, inputs resident in HBM,
-L2 flushed between steps, device-timed with CUDA events. The metric is
-algorithmic TFLOP/s (attended pairs only: fwd 4*d*P, fwd+bwd 14*d*P).
+forward, gated backward with dS) on the long-context training workload
+B=1, Hq=32, Hkv=8, d=128, N=32768 (512 blocks), block 64, bf16, inputs
+resident in HBM, L2 flushed between steps, device-timed with CUDA events. The
+metric is algorithmic TFLOP/s (attended pairs only: fwd 4*d*P, fwd+bwd
+14*d*P). The N=8192 training step, the sparse prefill and the decode are
+reported under "extra".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -35,7 +37,7 @@ from gated_block_sparse_gate_b200.inputs import WORKLOADS, make_decode_inputs, m
 
 METRIC = "gated sparse attention TFLOP/s (fwd+bwd and fwd) and % of bf16 tensor peak"
 UNIT = "TFLOP/s"
-HEADLINE = "train_bf16_n8192"
+HEADLINE = "train_bf16_n32768"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 
@@ -53,6 +55,25 @@ def sparse_pairs_per_head(Nb: int, bs: int, k: int) -> int:
     return bs * bs * hist + Nb * bs * (bs + 1) // 2
 
 
+def decode_union_blocks(S, cur: int, k: int, G: int) -> int:
+    """Distinct K/V blocks one decode step must read: per (sequence, kv group),
+    the union of its q-heads' Top-K historical blocks, plus the current block.
+
+    S is the per-q-head score tensor [B, Hq, Nb] (on any device); selection
+    follows the decode's rule (the k largest scores among blocks 0 .. cur-1).
+    Byte accounting only: which rows tie is irrelevant to the count for these
+    continuous scores."""
+    B, Hq = S.shape[:2]
+    kk = min(k, cur)
+    n_groups = B * (Hq // G)
+    if kk == 0:
+        return n_groups
+    top = torch.topk(S[..., :cur], kk, dim=-1).indices
+    mark = torch.zeros(B, Hq // G, cur, dtype=torch.bool, device=S.device)
+    mark.scatter_(2, top.reshape(B, Hq // G, G * kk), True)
+    return int(mark.sum().item()) + n_groups
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -63,16 +84,17 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def traffic_for(kernel: str):
+def traffic_for(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if still current.
 
-    profiles/traffic.json maps a kernel name to the bytes measured by ncu and the
-    SHA-256 of the source file it was measured from; a changed source voids it.
+    profiles/traffic.json maps "kernel/workload" to the bytes ncu measured for
+    one launch on that workload and the SHA-256 of the source file it was
+    measured from; a changed source voids it.
     """
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            entry = json.load(f)[kernel]
+            entry = json.load(f)[f"{kernel}/{workload}"]
         src = os.path.join(ROOT, entry["source"])
         with open(src, "rb") as f:
             if hashlib.sha256(f.read()).hexdigest() != entry["sha256"]:
@@ -208,7 +230,7 @@ def bench_training(w, steps, warmup, rank, dev, peaks):
     }
     dom = max(kern, key=lambda n: kern[n]["ms"])
     ach = kern[dom]["flops"] / (kern[dom]["ms"] * 1e-3) / 1e12
-    tr = traffic_for(dom)
+    tr = traffic_for(dom, w.name)
     roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": peaks["bf16_tflops"],
             "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
             "traffic": tr, "traffic_unit": "bytes per launch",
@@ -263,17 +285,38 @@ def bench_training(w, steps, warmup, rank, dev, peaks):
     t_end.record(s_out)
     torch.cuda.synchronize()
     e_ms = t_start.elapsed_time(t_end) / e_steps
+    # One call on its own: copy in, compute, copy out, on one stream, nothing
+    # overlapped (the latency a single step through the API costs).
+    bf = bufs[0]
+    serial = []
+    for k in range(max(3, min(steps, 10))):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        for n in names:
+            bf[n].copy_(host_in[n], non_blocking=True)
+        gb.forward(bf["Q"], bf["K"], bf["V"], bf["S"], mode="train", out=bf["O"], lse=bf["LSE"],
+                   ws=ws_f)
+        gb.backward(bf["Q"], bf["K"], bf["V"], bf["S"], bf["O"], bf["LSE"], bf["dO"],
+                    grads=bf["grads"], ws=ws_b)
+        for h, t in zip(host_out[0], (bf["O"], bf["LSE"], *bf["grads"])):
+            h.copy_(t, non_blocking=True)
+        b.record()
+        torch.cuda.synchronize()
+        if k > 0:  # the first call warms the copy paths
+            serial.append(a.elapsed_time(b))
     res["e2e"] = {"ms": e_ms, "h2d": sum(t.numel() * t.element_size() for t in host_in.values()),
                   "d2h": sum(t.numel() * t.element_size() for t in host_out[0]),
-                  "pipelined": "two buffer sets; the copies of steps k+1 and k-1 overlap step k"}
+                  "pipelined": "two buffer sets; the copies of steps k+1 and k-1 overlap step k",
+                  "serial_ms": statistics.mean(serial)}
     return res
 
 
-def bench_training_long(dev, peaks, reps=5):
-    """Long-context training step (N=32768, 512 blocks): forward + backward."""
+def bench_training_extra(name, dev, peaks, reps=5):
+    """Another training workload's step: forward + backward kernel times."""
     from gated_block_sparse_gate_b200 import binding as gb
 
-    w = WORKLOADS["train_bf16_n32768"]
+    w = WORKLOADS[name]
     x = make_prefill_inputs(w)
     d = {k: v.to(dev) for k, v in x.items()}
     del x
@@ -290,7 +333,8 @@ def bench_training_long(dev, peaks, reps=5):
         gb.forward(Q, K, V, S, mode="train", out=O, lse=LSE, ws=ws_f)
         gb.backward(Q, K, V, S, O, LSE, dO, grads=grads, ws=ws_b)
 
-    for _ in range(2):
+    for _ in range(3):
+        flush.zero_()
         step()
     a0, a1 = _events(reps), _events(reps)
     f0, f1, b0, b1 = _events(reps), _events(reps), _events(reps), _events(reps)
@@ -428,13 +472,23 @@ def bench_decode(dev, peaks, reps=10):
     kms = statistics.mean(a.elapsed_time(b) for a, b in zip(k0, k1))
     cur = (w.N - 1) // w.block
     blocks = min(k, cur) + 1
-    kv_bytes = w.B * w.Hq * blocks * w.block * w.d * 2 * 2  # K and V per q-head selection
+    G = w.Hq // w.Hkv
+    blk_bytes = w.block * w.d * 2 * 2  # K and V rows of one 64-token block
+    # algorithmic bytes: each distinct block of a (sequence, kv group) once
+    union = decode_union_blocks(x["S"], cur, k, G)
+    kv_bytes = union * blk_bytes
+    # logical bytes: every q-head's own selection (blocks shared by the heads of
+    # a group are requested once per head; the repeats mostly hit L2)
+    kv_logical = w.B * w.Hq * blocks * blk_bytes
     other = x["q"].numel() * 2 * 2 + x["S"].numel() * 4
     tot = kv_bytes + other
     out = {"ms": ms, "kernel_ms": kms, "tokens_per_s": w.B / (ms * 1e-3),
            "hbm_gbs": tot / (ms * 1e-3) / 1e9, "kernel_hbm_gbs": kv_bytes / (kms * 1e-3) / 1e9,
            "frac_of_hbm_roofline": (tot / (peaks["hbm_gbs"] * 1e9)) / (ms * 1e-3),
-           "bytes_per_step": tot}
+           "bytes_per_step": tot, "kv_union_blocks": union,
+           "bytes_note": "union of the selected blocks per (sequence, kv group) + q, O, S",
+           "logical_bytes_per_q_head": kv_logical + other,
+           "kernel_logical_gbs_per_q_head": kv_logical / (kms * 1e-3) / 1e9}
 
     def timed(call):
         for _ in range(3):
@@ -478,23 +532,46 @@ def bench_decode(dev, peaks, reps=10):
     torch.cuda.empty_cache()
     pms, pkms = timed(lambda: gb.decode_ex(x["q"], pools[0], pools[1], x["S"], w.N, topk=k,
                                             block_table=table, out=O, lse=LSE, ws=ws))
+    p_tot = tot + table.numel() * 4
     out["paged"] = {"ms": pms, "kernel_ms": pkms, "tokens_per_s": w.B / (pms * 1e-3),
-                    "hbm_gbs": tot / (pms * 1e-3) / 1e9,
-                    "frac_of_hbm_roofline": (tot / (peaks["hbm_gbs"] * 1e9)) / (pms * 1e-3),
-                    "bytes_per_step": tot + table.numel() * 4}
+                    "hbm_gbs": p_tot / (pms * 1e-3) / 1e9,
+                    "frac_of_hbm_roofline": (p_tot / (peaks["hbm_gbs"] * 1e9)) / (pms * 1e-3),
+                    "bytes_per_step": p_tot}
     del x, pools
     torch.cuda.empty_cache()
     return out
 
 
-def cpu_baseline_sample(w, min_s=10.0):
+def prefix_inputs(w, max_tokens):
+    """The workload's seeded inputs cut to their first ``max_tokens`` tokens
+    (query blocks 0 .. max_tokens/64 - 1 and the keys they attend: a causal
+    prefix computes exactly what those rows compute in the full problem).
+    Returns (inputs, workload with N = the prefix length)."""
+    import dataclasses
+
+    x = make_prefill_inputs(w)
+    if w.N <= max_tokens:
+        return x, w
+    nb = max_tokens // w.block
+    x = {k: (v[:, :, :max_tokens] if k != "S" else v[:, :, :nb, :nb]).contiguous()
+         for k, v in x.items()}
+    return x, dataclasses.replace(w, N=max_tokens)
+
+
+def cpu_baseline_sample(w, min_s=10.0, max_tokens=8192):
     """The float64 oracle on whole kv groups (G q-heads each) of the training
-    workload, group after group until at least ``min_s`` seconds are timed."""
+    workload, group after group until at least ``min_s`` seconds are timed.
+
+    Workloads longer than ``max_tokens`` are sampled on their first
+    ``max_tokens`` tokens (query blocks 0 .. max_tokens/64 - 1 with the keys
+    they attend, a causal prefix of the same seeded inputs), so the sample
+    stays within tens of seconds of CPU work."""
     import numpy as np
 
     import oracle
 
-    x = make_prefill_inputs(w)
+    n_full = w.N
+    x, w = prefix_inputs(w, max_tokens)
     G = w.Hq // w.Hkv
     f64 = lambda t: t.float().numpy().astype(np.float64)  # noqa: E731
     dt, groups = 0.0, 0
@@ -518,8 +595,9 @@ def cpu_baseline_sample(w, min_s=10.0):
     return {"value": fl / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"float64 NumPy oracle, forward+backward of "
                       f"{'kv group 0' if groups == 1 else f'kv groups 0-{groups - 1}'} "
-                      f"({groups * G} of {w.Hq} q-heads) of {w.name}; {dt:.1f} s; "
-                      f"host cores {os.cpu_count()}"}
+                      f"({groups * G} of {w.Hq} q-heads) of {w.name}"
+                      + (f", first {w.N} of {n_full} tokens" if n_full != w.N else "")
+                      + f"; {dt:.1f} s; host cores {os.cpu_count()}"}
 
 
 # -------------------------------------------------------------- reference arm
@@ -533,10 +611,12 @@ def run_reference(args, w):
     rank, _, ws = gdist.world()
     if rank != 0:
         return 0
-    n_sub = 2048  # prefix sub-problem of the same workload: one kv-group, N' = 2048
-    x = make_prefill_inputs(w, N=n_sub, Hq=w.Hq // w.Hkv, Hkv=1)
+    n_sub = 2048  # kv group 0 (q-heads 0-3) over the first 2048 tokens of the workload
+    x, _ = prefix_inputs(w, n_sub)
+    G = w.Hq // w.Hkv
     f64 = lambda t: t.float().numpy().astype(np.float64)  # noqa: E731
-    Q, K, V, dO, S = f64(x["Q"]), f64(x["K"]), f64(x["V"]), f64(x["dO"]), x["S"].numpy()
+    Q, dO, S = f64(x["Q"][:, :G]), f64(x["dO"][:, :G]), x["S"][:, :G].numpy()
+    K, V = f64(x["K"][:, :1]), f64(x["V"][:, :1])
 
     def step():
         oracle.gated_attention_forward(Q, K, V, S, w.block)
@@ -548,10 +628,10 @@ def run_reference(args, w):
     for _ in range(args.steps):
         step()
     dt = (time.perf_counter() - t0) / args.steps
-    fl = 14.0 * w.d * train_pairs_per_head(n_sub // w.block, w.block) * (w.Hq // w.Hkv)
+    fl = 14.0 * w.d * train_pairs_per_head(n_sub // w.block, w.block) * G
     val = fl / dt / 1e12
-    sample = (f"float64 NumPy oracle, forward+backward of one kv-group (4 q-heads) of a "
-              f"{n_sub}-token prefix of {w.name} per step")
+    sample = (f"float64 NumPy oracle, forward+backward of kv group 0 ({G} q-heads) over the "
+              f"first {n_sub} of {w.N} tokens of {w.name} per step")
     line = {"metric": METRIC, "value": val, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -606,7 +686,7 @@ def main(argv=None):
     e2e_ms = gdist.max_over_ranks(r["e2e"]["ms"], dev)
     extra = {}
     if ws == 1 and not args.no_extra:
-        extra["train_bf16_n32768"] = bench_training_long(dev, peaks)
+        extra["train_bf16_n8192"] = bench_training_extra("train_bf16_n8192", dev, peaks)
         extra["sparse_prefill_bf16_n65536"] = bench_sparse_prefill(dev, peaks)
         extra["sparse_decode_bf16_b64_l131072"] = bench_decode(dev, peaks)
     if rank == 0:
@@ -623,7 +703,9 @@ def main(argv=None):
             "roofline": r["roofline"],
             "e2e": {"value": total / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": r["e2e"]["h2d"], "d2h_bytes_per_step": r["e2e"]["d2h"],
-                    "ms_per_step": e2e_ms, "pipelined": r["e2e"]["pipelined"]},
+                    "ms_per_step": e2e_ms, "pipelined": r["e2e"]["pipelined"],
+                    "serial_ms_per_call": r["e2e"]["serial_ms"],
+                    "serial_value": total / (r["e2e"]["serial_ms"] * 1e-3) / 1e12},
             "gpu_launches": r["launches"], "gpu_launches_per_step": r["per_step_launches"],
             "clocks": r["clocks"],
         }

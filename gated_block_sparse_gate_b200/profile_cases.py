@@ -2,6 +2,7 @@
 
     python -m gated_block_sparse_gate_b200.profile_cases --case train_fwd --reps 3
     python -m gated_block_sparse_gate_b200.profile_cases --case train_bwd --reps 3
+    python -m gated_block_sparse_gate_b200.profile_cases --case train_bwd --workload train_bf16_n32768
     python -m gated_block_sparse_gate_b200.profile_cases --case sparse_fwd --topk 16 --reps 3
     python -m gated_block_sparse_gate_b200.profile_cases --case sparse_bwd --topk 16 --seq 16384
     python -m gated_block_sparse_gate_b200.profile_cases --case decode --batch 8 --reps 3
@@ -30,6 +31,7 @@ def main(argv=None):
     ap.add_argument("--seq", type=int, default=None, help="override N (prefill) or L (decode)")
     ap.add_argument("--batch", type=int, default=None, help="override B (decode)")
     ap.add_argument("--topk", type=int, default=None)
+    ap.add_argument("--workload", default=None, help="training workload (default train_bf16_n8192)")
     args = ap.parse_args(argv)
     build()
     gb.load_library()
@@ -50,7 +52,8 @@ def main(argv=None):
                          group_shared=args.case == "decode_grouped")
     else:
         sparse = args.case in ("sparse_fwd", "sparse_bwd")
-        w = WORKLOADS["sparse_prefill_bf16_n65536" if sparse else "train_bf16_n8192"]
+        w = WORKLOADS["sparse_prefill_bf16_n65536" if sparse else
+                      (args.workload or "train_bf16_n8192")]
         if args.seq:
             w = dataclasses.replace(w, N=args.seq)
         bwd = args.case in ("train_bwd", "sparse_bwd")

@@ -23,8 +23,42 @@ def test_pair_counts_match_the_oracle(Nb, k):
 
 
 def test_headline_pair_count():
-    """train_bf16_n8192: 1.0739e9 attended pairs over the 32 heads (FLOP basis)."""
+    """train_bf16_n8192: 1.0739e9 attended pairs over the 32 heads (FLOP basis);
+    train_bf16_n32768 (the headline): 1.7180e10."""
     assert bench.train_pairs_per_head(128, 64) * 32 == 1073872896  # 64*64*(128*127/2) + 128*(64*65/2), x 32
+    assert bench.train_pairs_per_head(512, 64) * 32 == 17180393472  # 64*64*(512*511/2) + 512*(64*65/2), x 32
+
+
+def test_decode_union_blocks_against_sets():
+    """Decode bytes count each distinct block of a (sequence, kv group) once:
+    the count equals the size of the union of the group's per-head Top-K sets
+    (oracle selection) plus one current block per group."""
+    import torch
+    rng = np.random.default_rng(5)
+    for B, Hq, G, Nb, k in ((3, 8, 4, 40, 6), (2, 4, 1, 17, 5), (1, 6, 3, 9, 20), (2, 4, 2, 12, 0)):
+        S = rng.standard_normal((B, Hq, Nb)) * math.sqrt(2)
+        cur = Nb - 1
+        want = 0
+        for b in range(B):
+            for g in range(Hq // G):
+                u = set()
+                for h in range(g * G, (g + 1) * G):
+                    u |= set(oracle.attended_blocks(S[b, h], cur, oracle.SPARSE, k).tolist())
+                want += len(u) + 1
+        assert bench.decode_union_blocks(torch.as_tensor(S), cur, k, G) == want
+
+
+def test_prefix_inputs_are_the_workload_prefix():
+    """The CPU samples read the first tokens of the workload's own inputs."""
+    from gated_block_sparse_gate_b200.inputs import WORKLOADS, make_prefill_inputs
+    import dataclasses
+    w = dataclasses.replace(WORKLOADS["train_bf16_n8192"], N=1024)
+    full = make_prefill_inputs(w)
+    x, wp = bench.prefix_inputs(w, 256)
+    assert wp.N == 256 and wp.Nb == 4
+    for k in ("Q", "K", "V", "dO"):
+        assert np.array_equal(x[k].float().numpy(), full[k][:, :, :256].float().numpy())
+    assert np.array_equal(x["S"].numpy(), full["S"][:, :, :4, :4].numpy())
 
 
 def test_traffic_is_tied_to_the_measured_source(tmp_path, monkeypatch):
@@ -32,13 +66,14 @@ def test_traffic_is_tied_to_the_measured_source(tmp_path, monkeypatch):
     src.write_text("// kernel v1\n")
     digest = hashlib.sha256(src.read_bytes()).hexdigest()
     (tmp_path / "profiles").mkdir()
-    table = {"k": {"source": "k.cu", "sha256": digest, "bytes_per_launch": 12345}}
+    table = {"k/w1": {"source": "k.cu", "sha256": digest, "bytes_per_launch": 12345}}
     (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(table))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.traffic_for("k") == 12345.0
-    assert bench.traffic_for("missing") is None
+    assert bench.traffic_for("k", "w1") == 12345.0
+    assert bench.traffic_for("k", "w2") is None  # measured on another workload
+    assert bench.traffic_for("missing", "w1") is None
     src.write_text("// kernel v2\n")  # the kernel changed since the counters were taken
-    assert bench.traffic_for("k") is None
+    assert bench.traffic_for("k", "w1") is None
 
 
 def _union_tiling_fraction(S, k):
@@ -113,4 +148,4 @@ def test_reference_arm_prints_the_contract_line(capsys):
     assert line["impl"] == "reference" and line["value"] > 0 and line["steps"] == 1
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["unit"] == line["unit"]
-    assert line["config"]["workload"] == "train_bf16_n8192"
+    assert line["config"]["workload"] == "train_bf16_n32768"
