@@ -30,7 +30,6 @@ namespace {
 
 constexpr size_t kScratchBytes = GBS_DECODE_NOALLOC_SCRATCH_BYTES;
 constexpr int kMaxDevices = 64;
-constexpr int kMaxSplitsNoalloc = 8;
 
 __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
@@ -76,69 +75,51 @@ extern "C" gbs_status gbs_decode_noalloc(const gbs_params* in, const void* q, co
                                          const void* Vc, const float* S, void* O, float* LSE,
                                          int num_splits, void* stream) {
   gbs::set_last_error("");
-  if (!in) return noalloc_fail(GBS_ERR_INVALID_ARG, "params is NULL");
-  const gbs_params& p = *in;
-  if (p.B <= 0 || p.Hq <= 0 || p.Hkv <= 0 || p.N <= 0 || p.Hq % p.Hkv)
-    return noalloc_fail(GBS_ERR_INVALID_ARG, "B, Hq, Hkv, N must be positive and Hq % Hkv == 0");
-  if (p.block != 64) return noalloc_fail(GBS_ERR_UNSUPPORTED, "block must be 64");
-  if (p.d != 64 && p.d != 128) return noalloc_fail(GBS_ERR_UNSUPPORTED, "d must be 64 or 128");
-  if (p.dtype != GBS_BF16 && p.dtype != GBS_F32) return noalloc_fail(GBS_ERR_INVALID_ARG, "unknown dtype");
-  if (p.topk < 0 || p.topk > GBS_MAX_TOPK) return noalloc_fail(GBS_ERR_INVALID_ARG, "topk out of range");
-  if (!(p.scale >= 0.f) || isinf(p.scale)) return noalloc_fail(GBS_ERR_INVALID_ARG, "bad scale");
-  const bool threshold = p.mode == GBS_THRESHOLD;
-  if (threshold && !(p.tau > 0.f && p.tau <= 1.f))
-    return noalloc_fail(GBS_ERR_INVALID_ARG, "threshold mode needs 0 < tau <= 1");
-  if (num_splits < 0 || num_splits > kMaxSplitsNoalloc)
-    return noalloc_fail(GBS_ERR_INVALID_ARG, "num_splits must be in [0, 8]");
+  // the same validation as gbs_decode (shape, mode, dtype, size limits)
+  gbs::Problem pr{};
+  gbs_status s = gbs::resolve_params(in, GBS_OP_DECODE, &pr);
+  if (s != GBS_OK) return s;
+  if (num_splits < 0 || num_splits > gbs::kMaxDecodeSplits)
+    return noalloc_fail(GBS_ERR_INVALID_ARG, "num_splits must be in [0, 32]");
   const void* ptrs[] = {q, Kc, Vc, S, O, LSE};
   for (const void* ptr : ptrs)
     if (!ptr || ((uintptr_t)ptr & 15u))
       return noalloc_fail(GBS_ERR_INVALID_ARG, "a tensor pointer is NULL or not 16-byte aligned");
 
-  gbs::Problem pr;
-  pr.B = p.B; pr.Hq = p.Hq; pr.Hkv = p.Hkv; pr.N = p.N; pr.d = p.d; pr.bs = p.block;
-  pr.Nb = (p.N + p.block - 1) / p.block; pr.G = p.Hq / p.Hkv; pr.topk = p.topk;
-  pr.mode = threshold ? GBS_THRESHOLD : GBS_SPARSE; pr.dtype = p.dtype;
-  pr.log_tau = threshold ? logf(p.tau) : 0.f;
-  pr.scale = p.scale > 0.f ? p.scale : 1.0f / sqrtf((float)p.d);
-  pr.scale_log2 = pr.scale * GBS_LOG2E;
-
-  const size_t rows = (size_t)p.B * p.Hq;
-  const int cur = (p.N - 1) / p.block;
-  const int n_ent = (p.topk < cur ? p.topk : cur) + 1;
+  const size_t rows = (size_t)pr.B * pr.Hq;
+  const int cur = (pr.N - 1) / pr.bs;
+  const int n_ent = (pr.topk < cur ? pr.topk : cur) + 1;
   int splits = num_splits;
   if (splits == 0) {
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    splits = (int)((2 * (size_t)sms * 16 + rows - 1) / rows);
-    if (splits > kMaxSplitsNoalloc) splits = kMaxSplitsNoalloc;
-    while (splits > 1 && scratch_needed(rows, p.topk, splits, p.d) > kScratchBytes) --splits;
+    // gbs_decode's rule, stepped down only if its partials would not fit
+    cudaError_t e = gbs::decode_auto_splits(pr, false, n_ent, &splits);
+    if (e != cudaSuccess) return noalloc_fail(GBS_ERR_CUDA, cudaGetErrorString(e));
+    while (splits > 1 && scratch_needed(rows, pr.topk, splits, pr.d) > kScratchBytes) --splits;
   }
   if (splits > n_ent) splits = n_ent;
   if (splits < 1) splits = 1;
-  if (scratch_needed(rows, p.topk, splits, p.d) > kScratchBytes)
+  if (scratch_needed(rows, pr.topk, splits, pr.d) > kScratchBytes)
     return noalloc_fail(GBS_ERR_INVALID_ARG,
                         "B*Hq, topk, splits and d need more than the static scratch "
                         "(GBS_DECODE_NOALLOC_SCRATCH_BYTES); use gbs_decode with a workspace");
 
   void* base = nullptr;
-  gbs_status s = scratch_address(&base);
+  s = scratch_address(&base);
   if (s != GBS_OK) return s;
   char* c = static_cast<char*>(base);
   gbs::Selection sel{};
   sel.idx = reinterpret_cast<int32_t*>(c);
-  c += align256(rows * p.topk * sizeof(int32_t));
+  c += align256(rows * pr.topk * sizeof(int32_t));
   sel.cnt = reinterpret_cast<int32_t*>(c);
   c += align256(rows * sizeof(int32_t));
   sel.logg = reinterpret_cast<float*>(c);
-  c += align256(rows * p.topk * sizeof(float));
+  c += align256(rows * pr.topk * sizeof(float));
   float* part_ml = reinterpret_cast<float*>(c);
   c += align256(rows * splits * 2 * sizeof(float));
   float* part_acc = reinterpret_cast<float*>(c);
 
   cudaStream_t st = (cudaStream_t)stream;
-  cudaError_t e = gbs::launch_select(S, (int)rows, pr.Nb, 1, cur, p.topk, pr.mode, pr.log_tau,
+  cudaError_t e = gbs::launch_select(S, (int)rows, pr.Nb, 1, cur, pr.topk, pr.mode, pr.log_tau,
                                      sel.idx, sel.cnt, sel.logg, nullptr, st);
   if (e == cudaSuccess)
     e = gbs::launch_decode(pr, q, Kc, Vc, sel, splits, part_ml, part_acc, O, LSE, st,

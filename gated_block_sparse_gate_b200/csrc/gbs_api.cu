@@ -34,7 +34,7 @@ gbs_status cuda_status(cudaError_t e, const char* where) {
 }
 
 constexpr size_t kAlign = 256;
-constexpr int kMaxSplits = 32;
+constexpr int kMaxSplits = kMaxDecodeSplits;
 inline size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 // Workspace carving: [header | regions...], each region 256-byte aligned.
@@ -80,8 +80,10 @@ FwdWs carve_fwd(const Problem& p, void* ws) {
     w.sel.idx = c.take<int32_t>(rows * p.topk);
     w.sel.cnt = c.take<int32_t>(rows);
     w.sel.logg = c.take<float>(rows * p.topk);
-    const size_t tiles = (size_t)p.B * p.Hq * ((p.Nb + 1) / 2);
-    w.plan = c.take<int32_t>(tiles * plan_stride(p) * 3);
+    if (!fwd_tq_supported(p)) {  // the paired-tile kernel's slot plan
+      const size_t tiles = (size_t)p.B * p.Hq * ((p.Nb + 1) / 2);
+      w.plan = c.take<int32_t>(tiles * plan_stride(p) * 3);
+    }
   }
   w.bytes = c.off;
   return w;
@@ -182,6 +184,29 @@ unsigned int* err_word(void* ws) { return reinterpret_cast<unsigned int*>(ws); }
 
 namespace gbs {
 void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+gbs_status resolve_params(const gbs_params* in, int op, Problem* out) { return resolve(in, op, out); }
+
+cudaError_t decode_auto_splits(const Problem& p, bool grouped, int n_ent, int* splits) {
+  // Shares of at most 17 blocks per CTA, and at least two waves of the split
+  // kernel's resident CTAs. On the 64 x 131072, K = 32 decode both variants
+  // are fastest at 2 splits (16-17 blocks a CTA): per q-head row 0.363 ms
+  // against 0.375 / 0.373 ms at 1 / 3; per shared-selection row 0.175 ms
+  // against 0.179 ms at 3 and 0.187 ms at 6.
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int cta_rows = grouped ? p.B * p.Hkv * (p.G / decode_heads_per_cta(p, true)) : p.B * p.Hq;
+  const int two_waves = 2 * sms * decode_resident_ctas(p, grouped);
+  const int by_share = (n_ent + 16) / 17;
+  const int by_waves = (two_waves + cta_rows - 1) / cta_rows;
+  int s = by_share > by_waves ? by_share : by_waves;
+  if (s > n_ent) s = n_ent;
+  if (s > kMaxSplits) s = kMaxSplits;
+  if (s < 1) s = 1;
+  *splits = s;
+  return cudaSuccess;
+}
 void note_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 void timer_begin(int op, cudaStream_t st) {
   if (g_timer[op][0]) cudaEventRecord(g_timer[op][0], st);
@@ -282,6 +307,10 @@ gbs_status gbs_fwd(const gbs_params* in, const void* Q, const void* K, const voi
   if (e != cudaSuccess) return cuda_status(e, "gbs_fwd/select");
   if (fwd_tc2_supported(p)) {
     e = launch_fwd_tc2(p, Q, K, V, S, w.sel.slse, O, LSE, err_word(ws), st);
+    if (e != cudaErrorNotSupported) return cuda_status(e, "gbs_fwd/attention");
+  }
+  if (fwd_tq_supported(p)) {
+    e = launch_fwd_tq(p, Q, K, V, w.sel, O, LSE, err_word(ws), st);
     if (e != cudaErrorNotSupported) return cuda_status(e, "gbs_fwd/attention");
   }
   if (p.dtype == GBS_BF16 && fwd_tc_supported(p)) {
@@ -386,21 +415,10 @@ gbs_status gbs_decode_ex(const gbs_params* in, const gbs_kv_layout* kvl, const v
                                 nullptr, 0, seq);
   if (e != cudaSuccess) return cuda_status(e, "gbs_decode/select");
   const int n_ent = (p.topk < cur_max ? p.topk : cur_max) + 1;
-  const int cta_rows = grouped ? p.B * p.Hkv * (p.G / decode_heads_per_cta(p, true)) : p.B * p.Hq;
   int splits = num_splits;
   if (splits == 0) {
-    // Shares of at most 17 blocks per CTA, and at least two waves of the split
-    // kernel's resident CTAs. On the 64 x 131072, K = 32 decode both variants
-    // are fastest at 2 splits (16-17 blocks a CTA): per q-head row 0.363 ms
-    // against 0.375 / 0.373 ms at 1 / 3; per shared-selection row 0.175 ms
-    // against 0.179 ms at 3 and 0.187 ms at 6.
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int two_waves = 2 * sms * decode_resident_ctas(p, grouped);
-    const int by_share = (n_ent + 16) / 17;
-    const int by_waves = (two_waves + cta_rows - 1) / cta_rows;
-    splits = by_share > by_waves ? by_share : by_waves;
+    e = decode_auto_splits(p, grouped, n_ent, &splits);
+    if (e != cudaSuccess) return cuda_status(e, "gbs_decode/splits");
   }
   if (splits > n_ent) splits = n_ent;
   if (splits > kMaxSplits) splits = kMaxSplits;

@@ -25,6 +25,16 @@ struct Problem {
   float log_tau;      // threshold mode: ln(tau); 0 otherwise
 };
 
+// Validates a parameter block for one op (GBS_OP_FWD / BWD / DECODE) and
+// resolves it; on failure sets gbs_last_error() and returns the status.
+gbs_status resolve_params(const gbs_params* in, int op, Problem* out);
+// Most decode splits a call can ask for.
+constexpr int kMaxDecodeSplits = 32;
+// The decode's automatic split count for n_ent blocks per selection row:
+// the larger of "at most 17 blocks per CTA" and "two waves of resident CTAs",
+// clamped to [1, min(n_ent, kMaxDecodeSplits)].
+cudaError_t decode_auto_splits(const Problem& p, bool grouped, int n_ent, int* splits);
+
 // Selection buffers produced by K1 and read by the attention kernels.
 struct Selection {
   float* slse;     // [B, Hq, Nb]   training normaliser (may be null in sparse mode)
@@ -97,6 +107,13 @@ cudaError_t launch_fwd_tc2(const Problem& p, const void* Q, const void* K, const
                            const float* S, const float* slse, void* O, float* LSE,
                            unsigned int* err, cudaStream_t st);
 bool fwd_tc2_supported(const Problem& p);
+// Sparse / threshold mode, bf16, d = 128: one 64-query block per CTA with its
+// attended keys on the TMEM lanes (S^T = K Q^T, O^T += V^T P^T), reading K1's
+// lists directly (no plan).
+cudaError_t launch_fwd_tq(const Problem& p, const void* Q, const void* K, const void* V,
+                          const Selection& sel, void* O, float* LSE, unsigned int* err,
+                          cudaStream_t st);
+bool fwd_tq_supported(const Problem& p);
 // Per-(batch, head, 128-row tile) slot plan of sparse mode (union of the tile's
 // two query blocks' Top-K lists plus their current blocks, with per-half biases).
 cudaError_t launch_plan(const Problem& p, const Selection& sel, int32_t* plan, int plan_stride,
@@ -113,6 +130,18 @@ cudaError_t launch_bwd_tc(const Problem& p, const void* Q, const void* K, const 
                           unsigned int* err, cudaStream_t st);
 bool bwd_tc_supported(const Problem& p);
 size_t bwd_plan_ints(const Problem& p);
+// Sparse / threshold backward, bf16, d = 128: one 64-key block per CTA over the
+// (q-head, query block) entries of its kv group that keep it (their plan is
+// built into `plan`, bwd_kb_plan_ints(p) ints). Dvec, the zeroed dQacc and Gblk
+// and the kept-set normaliser `slse` come from the caller; dQ conversion and
+// dS follow it.
+cudaError_t launch_bwd_kb(const Problem& p, const void* Q, const void* K, const void* V,
+                          const float* S, const float* slse, const float* LSE, const void* dO,
+                          void* dK, void* dV, const float* Dvec, float* Gblk, float* dQacc,
+                          const uint32_t* mbits, int mwords, int32_t* plan, unsigned int* err,
+                          cudaStream_t st);
+bool bwd_kb_supported(const Problem& p);
+size_t bwd_kb_plan_ints(const Problem& p);
 // dS from the tile sums G (shared by both backward paths); mbits as above.
 cudaError_t launch_ds_finalize(const Problem& p, const float* S, const float* slse,
                                const float* Gblk, float* dS, const uint32_t* mbits, int mwords,
