@@ -16,14 +16,14 @@ LIB_PATH = os.path.join(HERE, "libgbs.so")
 
 GBS_OK = 0
 STATUS_NAMES = {0: "GBS_OK", 1: "GBS_ERR_INVALID_ARG", 2: "GBS_ERR_UNSUPPORTED", 3: "GBS_ERR_CUDA",
-                4: "GBS_ERR_TIMEOUT", 5: "GBS_ERR_WORKSPACE"}
+                4: "GBS_ERR_TIMEOUT", 5: "GBS_ERR_WORKSPACE", 6: "GBS_ERR_DEVICE_CHECK"}
 MODES = {"train": 0, "sparse": 1, "threshold": 2}
 DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 OP_FWD, OP_BWD, OP_DECODE = 0, 1, 2
 
 EXPORTED = ("gbs_version", "gbs_status_string", "gbs_last_error", "gbs_workspace_bytes",
             "gbs_clear_error", "gbs_check", "gbs_select", "gbs_fwd", "gbs_bwd", "gbs_decode",
-            "gbs_set_timer", "gbs_launch_count")
+            "gbs_set_timer", "gbs_launch_count", "gbs_selftest_wait_timeout")
 
 
 class GbsError(RuntimeError):
@@ -349,6 +349,23 @@ def check(ws, stream=None):
     """Raises GbsError if a kernel recorded a device-side error in ``ws``."""
     _device("gbs_check", "ws", ws)
     _check(load_library().gbs_check(_ptr(ws), _stream(stream)), "gbs_check")
+
+
+def clear_error(ws, stream=None):
+    """Clears the device error word of ``ws`` (asynchronous)."""
+    _device("gbs_clear_error", "ws", ws)
+    _check(load_library().gbs_clear_error(_ptr(ws), _stream(stream)), "gbs_clear_error")
+
+
+def selftest_wait_timeout(ws, limit_us, stream=None):
+    """gbs_selftest_wait_timeout: one bounded device wait that nothing releases;
+    after ``limit_us`` it records GBS_ERR_TIMEOUT in the error word of ``ws``."""
+    lib = load_library()
+    f = lib.gbs_selftest_wait_timeout
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_uint, ctypes.c_void_p]
+    _device("gbs_selftest_wait_timeout", "ws", ws)
+    _check(f(_ptr(ws), int(limit_us), _stream(stream)), "gbs_selftest_wait_timeout")
 
 
 def decode_noalloc(q, Kc, Vc, S, L=None, block=64, topk=32, scale=0.0, num_splits=0, out=None,

@@ -75,7 +75,9 @@ typedef enum gbs_status {
   GBS_ERR_UNSUPPORTED = 2,   /* valid, but not a configuration this build runs  */
   GBS_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed     */
   GBS_ERR_TIMEOUT = 4,       /* a device-side bounded wait expired (gbs_check)  */
-  GBS_ERR_WORKSPACE = 5      /* workspace missing or smaller than required      */
+  GBS_ERR_WORKSPACE = 5,     /* workspace missing or smaller than required      */
+  GBS_ERR_DEVICE_CHECK = 6   /* debug build only: a device-side index check
+                                failed (the access was clamped; gbs_check)    */
 } gbs_status;
 
 typedef enum gbs_mode { GBS_TRAIN = 0, GBS_SPARSE = 1, GBS_THRESHOLD = 2 } gbs_mode;
@@ -239,6 +241,18 @@ GBS_API gbs_status gbs_set_timer(int op, void* start, void* stop);
 /* Total number of CUDA kernels this library has launched in this process. */
 GBS_API uint64_t gbs_launch_count(void);
 
+/* Failure-detection self-test (no counterpart in the paper). Launches one
+ * thread that waits, through the same bounded mbarrier wait every pipeline
+ * stage of the tensor-core kernels uses, on a shared-memory barrier that
+ * nothing arrives at. After limit_us microseconds (1 .. 1,000,000) the wait
+ * gives up, GBS_ERR_TIMEOUT is recorded in the error word of `ws` (its first
+ * 4 bytes; any device buffer of at least 256 bytes, 256-byte aligned) and the
+ * kernel returns; gbs_check(ws, stream) then reports it. Nothing traps or
+ * faults, so the CUDA context stays usable. Returns GBS_ERR_WORKSPACE or
+ * GBS_ERR_INVALID_ARG for a bad `ws` or limit, GBS_ERR_CUDA if the launch
+ * fails. */
+GBS_API gbs_status gbs_selftest_wait_timeout(void* ws, unsigned int limit_us, void* stream);
+
 /* Bytes of device scratch that gbs_decode_noalloc keeps in the library. */
 #define GBS_DECODE_NOALLOC_SCRATCH_BYTES (8u << 20)
 
@@ -254,9 +268,13 @@ GBS_API uint64_t gbs_launch_count(void);
  * array's address (cudaGetSymbolAddress, with the device current); make that
  * first call before any stream capture. Calls on one device share the array:
  * calls that overlap on the GPU race and must be serialised by the caller.
- * Rejects, with GBS_ERR_INVALID_ARG and a gbs_last_error() message, any size
- * whose scratch (about B*Hq*(8*topk + 8 + splits*(4*d + 8)) bytes, splits <= 8)
- * exceeds the array; allocates and frees nothing. */
+ * Validates its arguments exactly as gbs_decode does (same statuses). With
+ * num_splits = 0 it picks gbs_decode's split count, and so returns bitwise the
+ * same results, unless those partials would not fit the array, in which case
+ * it takes the largest count that fits. Rejects, with GBS_ERR_INVALID_ARG and a
+ * gbs_last_error() message, any size whose scratch (about
+ * B*Hq*(8*topk + 8 + splits*(4*d + 8)) bytes, splits <= 32) exceeds the array;
+ * allocates and frees nothing. */
 GBS_API gbs_status gbs_decode_noalloc(const gbs_params* p, const void* q, const void* Kc,
                                       const void* Vc, const float* S, void* O, float* LSE,
                                       int num_splits, void* stream);

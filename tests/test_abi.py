@@ -37,8 +37,8 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_version_and_status_strings(lib):
     assert lib.gbs_version() == (0 << 16) | 1
-    for s in range(6):
-        assert lib.gbs_status_string(s)
+    for s in range(7):
+        assert lib.gbs_status_string(s) != b"unknown status"
 
 
 def test_workspace_sizes(lib):
@@ -128,6 +128,37 @@ def test_decode_split_bounds(lib):
     ok = ctypes.c_void_p(4096)
     st = lib.gbs_decode(ctypes.byref(p), ok, ok, ok, ok, ok, ok, 999, ok, 1 << 30, None)
     assert st == 1
+
+
+@pytest.mark.parametrize("kw", [
+    dict(mode=7),                                   # unknown mode
+    dict(B=1024, Hq=64, Hkv=8, N=32768),            # 2^31 token rows: 32-bit cache row index
+    dict(d=96),                                     # head dim not built
+    dict(topk=10_000),                              # budget beyond the limit
+    dict(mode="threshold", tau=1.5),                # tau outside (0, 1]
+    dict(Hq=6, Hkv=4),                              # Hq not a multiple of Hkv
+])
+def test_noalloc_decode_rejects_what_decode_rejects(lib, kw):
+    """gbs_decode_noalloc validates exactly as gbs_decode does, before any
+    device call: same status for every invalid parameter block."""
+    args = dict(B=2, Hq=4, Hkv=2, N=1000, d=64, block=64, topk=4, mode="sparse", tau=0.0)
+    mode = kw.pop("mode", "sparse")
+    args.update(kw)
+    p = gb.make_params(**{**args, "mode": "sparse"})
+    p.mode = mode if isinstance(mode, int) else gb.MODES[mode]
+    ok = ctypes.c_void_p(4096)
+    lib.gbs_decode_noalloc.restype = ctypes.c_int
+    st_ws = lib.gbs_decode(ctypes.byref(p), ok, ok, ok, ok, ok, ok, 1, ok, 1 << 30, None)
+    st_na = lib.gbs_decode_noalloc(ctypes.byref(p), ok, ok, ok, ok, ok, ok, 1, None)
+    assert st_ws == st_na != 0, (st_ws, st_na, lib.gbs_last_error())
+
+
+def test_noalloc_decode_split_bounds(lib):
+    p = gb.make_params(2, 4, 2, 1000, 64, 64, 4, "sparse")
+    ok = ctypes.c_void_p(4096)
+    lib.gbs_decode_noalloc.restype = ctypes.c_int
+    for splits in (-1, 33):
+        assert lib.gbs_decode_noalloc(ctypes.byref(p), ok, ok, ok, ok, ok, ok, splits, None) == 1
 
 
 def test_binding_fails_loudly_without_library(tmp_path):
