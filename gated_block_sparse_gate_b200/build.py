@@ -1,7 +1,10 @@
 """Builds libgbs.so (all CUDA sources under csrc/) in-tree for sm_100a.
 
-Usage: python -m gated_block_sparse_gate_b200.build [--force]
-The library is rebuilt when any source or header is newer than it.
+Usage: python -m gated_block_sparse_gate_b200.build [--force] [--debug]
+The library is rebuilt when any source or header is newer than it. --debug
+builds libgbs_debug.so instead: the same sources with -DGBS_DEBUG, whose
+kernels check every index they read from a list and report a bad one as
+GBS_ERR_DEVICE_CHECK (a stand-in for a device memory checker).
 """
 from __future__ import annotations
 
@@ -15,6 +18,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libgbs.so")
+DEBUG_LIB = os.path.join(HERE, "libgbs_debug.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -28,27 +32,29 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale():
-    if not os.path.exists(LIB):
+def _stale(lib=LIB):
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) \
         + glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(f) > t for f in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    lib = DEBUG_LIB if debug else LIB
+    if not force and not _stale(lib):
+        return lib
     nvcc = os.environ.get("NVCC", "nvcc")
-    tmp = LIB + ".tmp"
-    cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
+    tmp = lib + ".tmp"
+    flags = NVCC_FLAGS + (["-DGBS_DEBUG"] if debug else [])
+    cmd = [nvcc, *flags, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
     if verbose:
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True))
+    print(build(force="--force" in sys.argv, verbose=True, debug="--debug" in sys.argv))

@@ -147,7 +147,7 @@ bwd_kb_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const int bk = (int)(blockIdx.x % BKV);
   const int b = bk / p.Hkv, kvh = bk % p.Hkv;
   const int32_t* list = a.plan + (size_t)blockIdx.x * a.plan_stride;
-  const int n_entries = __ldg(list);
+  const int n_entries = dcheck(__ldg(list), 0, p.G * (p.Nb - c), a.err);
   const int n_steps = (n_entries + 1) >> 1;
   // (batch x q-head row, query block) of entry i; r = -1 past the end
   auto entry_at = [&](int i, int& bh, int& r) {
@@ -155,8 +155,8 @@ bwd_kb_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     r = -1;
     if (i < n_entries) {
       const int e = __ldg(list + 1 + i);
-      hh = e >> 16;
-      r = e & 0xffff;
+      hh = dcheck(e >> 16, 0, p.G - 1, a.err);
+      r = dcheck(e & 0xffff, c, p.Nb - 1, a.err);
     }
     bh = b * p.Hq + kvh * p.G + hh;
   };

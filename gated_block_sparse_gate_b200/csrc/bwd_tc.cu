@@ -181,7 +181,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const int b = bk / p.Hkv, kvh = bk % p.Hkv;
   const int per_head = p.Nb - 2 * u;  // training: query blocks r >= 2u of each q-head
   const int32_t* list = a.plan ? a.plan + (size_t)blockIdx.x * a.plan_stride : nullptr;
-  const int n_entries = list ? __ldg(list) : p.G * per_head;
+  const int n_entries = list ? dcheck(__ldg(list), 0, p.G * per_head, a.err) : p.G * per_head;
   const int n_steps = (n_entries + 1) >> 1;
   // (batch x q-head row, query block) of list entry i; r = -1 past the end.
   // Step j takes entries 2j (query half 0) and 2j + 1 (query half 1).
@@ -191,8 +191,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     if (i < n_entries) {
       if (list) {
         const int e = __ldg(list + 1 + i);
-        hh = e >> 16;
-        r = e & 0xffff;
+        hh = dcheck(e >> 16, 0, p.G - 1, a.err);
+        r = dcheck(e & 0xffff, 2 * u, p.Nb - 1, a.err);
       } else {
         hh = i / per_head;
         r = 2 * u + i % per_head;

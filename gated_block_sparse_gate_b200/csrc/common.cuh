@@ -21,6 +21,24 @@ __device__ __forceinline__ void set_error(unsigned int* word, unsigned int code)
   if (word) atomicCAS(word, 0u, code);
 }
 
+// Device-side index checks of the debug build (compiled with -DGBS_DEBUG; the
+// library's stand-in for a memory checker). A value read from an index list
+// (a Top-K list, a count, a per-CTA plan) that lies outside [lo, hi] is
+// recorded as GBS_ERR_DEVICE_CHECK in the error word and replaced by lo, so the
+// access it would drive stays in bounds. Release builds compile it away.
+__device__ __forceinline__ int dcheck(int v, int lo, int hi, unsigned int* word) {
+#ifdef GBS_DEBUG
+  if (v < lo || v > hi) {
+    set_error(word, GBS_ERR_DEVICE_CHECK);
+    return lo;
+  }
+#endif
+  (void)lo;
+  (void)hi;
+  (void)word;
+  return v;
+}
+
 template <typename T> __device__ __forceinline__ float to_f32(T x);
 template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {

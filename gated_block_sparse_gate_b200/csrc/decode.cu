@@ -118,7 +118,7 @@ decode_split_kernel(Problem p, const T* __restrict__ q, const T* __restrict__ Kc
     L = L < 1 ? 1 : (L > p.N ? p.N : L);
   }
   const int cur = (L - 1) / kBS;
-  const int n_hist = sel.cnt[srow];
+  const int n_hist = dcheck(sel.cnt[srow], 0, min(p.topk, cur), kv.err);
   const int n_ent = n_hist + 1;  // + current block
   const int per = (n_ent + splits - 1) / splits;
   const int e0 = split * per, e1 = min(n_ent, e0 + per);
@@ -148,7 +148,7 @@ decode_split_kernel(Problem p, const T* __restrict__ q, const T* __restrict__ Kc
     for (int t = threadIdx.x; t < ce - cs; t += kThreads) {
       const int e = cs + t;
       const bool is_cur = e == n_hist;
-      const int c = is_cur ? cur : sel.idx[(size_t)srow * p.topk + e];
+      const int c = is_cur ? cur : dcheck(sel.idx[(size_t)srow * p.topk + e], 0, cur - 1, kv.err);
       int row0 = contig + c * kBS;
       if (kv.btab) {
         const int page = __ldg(kv.btab + (size_t)b * kv.max_blocks + c);

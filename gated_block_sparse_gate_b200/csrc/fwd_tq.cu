@@ -111,7 +111,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 // Entry e of the CTA's list: the selected blocks in K1's order, then the
 // current block (causal, bias 0), then one masked pad (current block again).
 __device__ __forceinline__ int entry_block(const TqArgs& a, size_t row, int r, int n_hist, int e) {
-  return e < n_hist ? __ldg(a.sel.idx + row * a.p.topk + e) : r;
+  return e < n_hist ? dcheck(__ldg(a.sel.idx + row * a.p.topk + e), 0, r - 1, a.err) : r;
 }
 
 __global__ void __launch_bounds__(kThreads, 2)
@@ -133,7 +133,7 @@ fwd_tq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
   const int b = bh / a.p.Hq, h = bh % a.p.Hq;
   const int kvz = b * a.p.Hkv + h / a.p.G;
   const size_t row = (size_t)bh * a.p.Nb + r;
-  const int n_hist = __ldg(a.sel.cnt + row);
+  const int n_hist = dcheck(__ldg(a.sel.cnt + row), 0, min(a.p.topk, r), a.err);
   const int n_stages = (n_hist + 2) / 2;  // n_hist + 1 entries, two per stage
 
   if (threadIdx.x == 0) {

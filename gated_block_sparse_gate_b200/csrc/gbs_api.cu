@@ -240,6 +240,7 @@ const char* gbs_status_string(gbs_status s) {
     case GBS_ERR_CUDA: return "CUDA error";
     case GBS_ERR_TIMEOUT: return "device wait timed out";
     case GBS_ERR_WORKSPACE: return "workspace missing or too small";
+    case GBS_ERR_DEVICE_CHECK: return "device index check failed (debug build)";
   }
   return "unknown status";
 }
