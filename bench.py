@@ -233,6 +233,8 @@ def bench_training(w, steps, warmup, rank, dev, peaks):
     tr = traffic_for(dom, w.name)
     roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": peaks["bf16_tflops"],
             "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
+            "peak_sustained": peaks["bf16_tflops_sustained"],
+            "frac_of_sustained": ach / peaks["bf16_tflops_sustained"],
             "traffic": tr, "traffic_unit": "bytes per launch",
             "flops_per_launch": kern[dom]["flops"], "launch_ms": kern[dom]["ms"]}
     res = dict(ms=ms, flops=fl_fb, fl_fwd=fl_fwd, launches=launches, clocks=clk, roofline=roof,

@@ -691,8 +691,7 @@ bool make_map_dq(CUtensorMap* m, const void* base, int d, size_t rows) {
 
 template <int D>
 cudaError_t launch_bwd_typed(const BwdArgs& a, const void* Q, const void* K, const void* V,
-                             const void* O, const void* dO, void* dQ, cudaStream_t st,
-                             bool key_block) {
+                             const void* O, const void* dO, void* dQ, cudaStream_t st) {
   const Problem& p = a.p;
   const size_t rows = (size_t)p.B * p.Hq * p.N;
   dot_rows_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
@@ -700,16 +699,6 @@ cudaError_t launch_bwd_typed(const BwdArgs& a, const void* Q, const void* K, con
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (key_block) {
-    e = launch_bwd_kb(p, Q, K, V, a.S, a.slse, a.LSE, dO, a.dK, a.dV, a.Dvec, a.Gblk, a.dQacc,
-                      a.mbits, a.mwords, const_cast<int32_t*>(a.plan), a.err, st);
-    if (e != cudaSuccess) return e;
-    const size_t n8 = rows * D / 8;
-    dq_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(a.dQacc, (__nv_bfloat16*)dQ,
-                                                                      p.scale, n8);
-    note_launch();
-    return cudaGetLastError();
-  }
   CUtensorMap tq, tk, tv, tdo, tdq, tq2, tdo2;
   if (!make_map128(&tq, Q, D, p.N, p.B * p.Hq, 64) || !make_map128(&tk, K, D, p.N, p.B * p.Hkv) ||
       !make_map128(&tv, V, D, p.N, p.B * p.Hkv) || !make_map128(&tdo, dO, D, p.N, p.B * p.Hq, 64) ||
@@ -742,7 +731,6 @@ bool bwd_tc_supported(const Problem& p) {
 
 size_t bwd_plan_ints(const Problem& p) {
   if (p.mode == GBS_TRAIN) return 0;
-  if (bwd_kb_supported(p)) return bwd_kb_plan_ints(p);
   const size_t n_tiles = (size_t)(p.Nb + 1) / 2;
   return (size_t)p.B * p.Hkv * n_tiles * (1 + (size_t)p.G * p.Nb);
 }
@@ -771,8 +759,7 @@ cudaError_t launch_bwd_tc(const Problem& p, const void* Q, const void* K, const 
   a.plan = sparse ? plan : nullptr;
   a.plan_stride = 1 + p.G * p.Nb;
   a.err = err;
-  const bool key_block = sparse && bwd_kb_supported(p);
-  if (sparse && !key_block) {
+  if (sparse) {
     const int ctas = p.B * p.Hkv * a.n_tiles;
     bwd_plan_kernel<<<(unsigned)((ctas + 7) / 8), 256, 0, st>>>(
         mbits, mwords, p.Nb, a.n_tiles, p.G, p.Hq, p.Hkv, p.B * p.Hkv, plan, a.plan_stride);
@@ -784,8 +771,8 @@ cudaError_t launch_bwd_tc(const Problem& p, const void* Q, const void* K, const 
   if (e == cudaSuccess)
     e = cudaMemsetAsync(Gblk, 0, (size_t)p.B * p.Hq * p.Nb * p.Nb * sizeof(float), st);
   if (e != cudaSuccess) return e;
-  if (p.d == 64) return launch_bwd_typed<64>(a, Q, K, V, O, dO, dQ, st, false);
-  return launch_bwd_typed<128>(a, Q, K, V, O, dO, dQ, st, key_block);
+  if (p.d == 64) return launch_bwd_typed<64>(a, Q, K, V, O, dO, dQ, st);
+  return launch_bwd_typed<128>(a, Q, K, V, O, dO, dQ, st);
 }
 
 }  // namespace gbs

@@ -80,10 +80,8 @@ FwdWs carve_fwd(const Problem& p, void* ws) {
     w.sel.idx = c.take<int32_t>(rows * p.topk);
     w.sel.cnt = c.take<int32_t>(rows);
     w.sel.logg = c.take<float>(rows * p.topk);
-    if (!fwd_tq_supported(p)) {  // the paired-tile kernel's slot plan
-      const size_t tiles = (size_t)p.B * p.Hq * ((p.Nb + 1) / 2);
-      w.plan = c.take<int32_t>(tiles * plan_stride(p) * 3);
-    }
+    const size_t tiles = (size_t)p.B * p.Hq * ((p.Nb + 1) / 2);
+    w.plan = c.take<int32_t>(tiles * plan_stride(p) * 3);
   }
   w.bytes = c.off;
   return w;
@@ -308,10 +306,6 @@ gbs_status gbs_fwd(const gbs_params* in, const void* Q, const void* K, const voi
   if (e != cudaSuccess) return cuda_status(e, "gbs_fwd/select");
   if (fwd_tc2_supported(p)) {
     e = launch_fwd_tc2(p, Q, K, V, S, w.sel.slse, O, LSE, err_word(ws), st);
-    if (e != cudaErrorNotSupported) return cuda_status(e, "gbs_fwd/attention");
-  }
-  if (fwd_tq_supported(p)) {
-    e = launch_fwd_tq(p, Q, K, V, w.sel, O, LSE, err_word(ws), st);
     if (e != cudaErrorNotSupported) return cuda_status(e, "gbs_fwd/attention");
   }
   if (p.dtype == GBS_BF16 && fwd_tc_supported(p)) {

@@ -107,13 +107,6 @@ cudaError_t launch_fwd_tc2(const Problem& p, const void* Q, const void* K, const
                            const float* S, const float* slse, void* O, float* LSE,
                            unsigned int* err, cudaStream_t st);
 bool fwd_tc2_supported(const Problem& p);
-// Sparse / threshold mode, bf16, d = 128: one 64-query block per CTA with its
-// attended keys on the TMEM lanes (S^T = K Q^T, O^T += V^T P^T), reading K1's
-// lists directly (no plan).
-cudaError_t launch_fwd_tq(const Problem& p, const void* Q, const void* K, const void* V,
-                          const Selection& sel, void* O, float* LSE, unsigned int* err,
-                          cudaStream_t st);
-bool fwd_tq_supported(const Problem& p);
 // Per-(batch, head, 128-row tile) slot plan of sparse mode (union of the tile's
 // two query blocks' Top-K lists plus their current blocks, with per-half biases).
 cudaError_t launch_plan(const Problem& p, const Selection& sel, int32_t* plan, int plan_stride,
@@ -130,18 +123,6 @@ cudaError_t launch_bwd_tc(const Problem& p, const void* Q, const void* K, const 
                           unsigned int* err, cudaStream_t st);
 bool bwd_tc_supported(const Problem& p);
 size_t bwd_plan_ints(const Problem& p);
-// Sparse / threshold backward, bf16, d = 128: one 64-key block per CTA over the
-// (q-head, query block) entries of its kv group that keep it (their plan is
-// built into `plan`, bwd_kb_plan_ints(p) ints). Dvec, the zeroed dQacc and Gblk
-// and the kept-set normaliser `slse` come from the caller; dQ conversion and
-// dS follow it.
-cudaError_t launch_bwd_kb(const Problem& p, const void* Q, const void* K, const void* V,
-                          const float* S, const float* slse, const float* LSE, const void* dO,
-                          void* dK, void* dV, const float* Dvec, float* Gblk, float* dQacc,
-                          const uint32_t* mbits, int mwords, int32_t* plan, unsigned int* err,
-                          cudaStream_t st);
-bool bwd_kb_supported(const Problem& p);
-size_t bwd_kb_plan_ints(const Problem& p);
 // dS from the tile sums G (shared by both backward paths); mbits as above.
 cudaError_t launch_ds_finalize(const Problem& p, const float* S, const float* slse,
                                const float* Gblk, float* dS, const uint32_t* mbits, int mwords,

@@ -66,9 +66,9 @@ def _prefill_run(x, mode, k, tau):
 
 
 @pytest.mark.parametrize("shape,mode,k,tau", [
-    ((2, 8, 2, 1024, 128), "sparse", 3, 0.0),      # transposed forward, key-block backward
+    ((2, 8, 2, 1024, 128), "sparse", 3, 0.0),      # slot plans and key-tile step lists
     ((1, 8, 2, 1024, 128), "threshold", 6, 0.05),
-    ((1, 4, 2, 448, 64), "sparse", 2, 0.0),         # paired-tile forward, key-tile backward lists
+    ((1, 4, 2, 448, 64), "sparse", 2, 0.0),         # d = 64, odd block count
     ((1, 8, 2, 1024, 128), "train", 0, 0.0),
 ])
 def test_debug_build_matches_release_and_reports_nothing(libs, shape, mode, k, tau):
