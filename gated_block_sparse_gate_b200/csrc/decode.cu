@@ -21,8 +21,12 @@
 // Serving layouts (gbs_decode_ex): the cache may sit on 64-token pages found
 // through a block table, each sequence may have its own length, and with
 // group-shared selection one CTA serves two q-heads of a kv group, so each
-// row it loads feeds both. A CTA resolves the addresses of up to 64 of its
-// blocks at once (index, gate, page) before it streams them.
+// row it loads feeds both. That variant is bound by instruction issue, not
+// bytes, so with d = 128 a lane's 16 dot-product partials (8 rows x 2 heads)
+// are reduced across its 16-lane group by one butterfly (15 shuffles), each
+// lane then takes one exponential, and the products run on packed fp32 pairs.
+// A CTA resolves the addresses of up to 64 of its blocks at once (index, gate,
+// page) before it streams them.
 #include "common.cuh"
 #include "internal.h"
 
@@ -70,6 +74,32 @@ __device__ __forceinline__ Vec8 load8<float>(const float* ptr) {
 __device__ __forceinline__ float bf16_elem(const uint4& u, int i) {
   const uint32_t w = i < 2 ? u.x : (i < 4 ? u.y : (i < 6 ? u.z : u.w));
   return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));
+}
+
+// packed fp32 pairs (one 64-bit register, two lanes of arithmetic per instruction)
+struct F2 { uint64_t v; };
+__device__ __forceinline__ F2 mk2(float lo, float hi) {
+  F2 r; asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "f"(lo), "f"(hi)); return r;
+}
+__device__ __forceinline__ F2 f2m(float a0, float a1, float b0, float b1) {
+  F2 r; asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(mk2(a0, a1).v), "l"(mk2(b0, b1).v)); return r;
+}
+__device__ __forceinline__ F2 f2fma(float a0, float a1, float b0, float b1, F2 c) {
+  F2 r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r.v) : "l"(mk2(a0, a1).v), "l"(mk2(b0, b1).v), "l"(c.v));
+  return r;
+}
+__device__ __forceinline__ float f2sum(F2 x) {
+  float lo, hi; asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x.v)); return lo + hi;
+}
+__device__ __forceinline__ void f2acc8(float (&acc)[8], float p, const float (&v)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    F2 r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r.v) : "l"(mk2(p, p).v), "l"(mk2(v[i], v[i + 1]).v),
+        "l"(mk2(acc[i], acc[i + 1]).v));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(acc[i]), "=f"(acc[i + 1]) : "l"(r.v));
+  }
 }
 
 // Online-softmax state of one lane group (log2 domain).
@@ -172,7 +202,88 @@ decode_split_kernel(Problem p, const T* __restrict__ q, const T* __restrict__ Kc
     // rows handled by this group inside the block
     const int row0 = group * ROWS_PER_GROUP;
     float s[NH][ROWS_PER_GROUP];
-    if constexpr (kRaw) {
+    if constexpr (kRaw && NH == 2 && LPK == 16) {
+      // bf16, two q-heads, 16 lanes a row: the 16 dot-product partials of a
+      // lane (8 rows x 2 heads) are reduced across the group by a butterfly that
+      // halves the values a lane keeps at offsets 8, 4, 2, 1, so lane `sub`
+      // ends with the full dot product of head sub / 8, row sub % 8 (15 shuffles
+      // instead of 16 four-level reductions). Each lane then takes one
+      // exponential; row maxima and sums reduce over the head's 8 lanes, and the
+      // PV update broadcasts each row's probability from its lane.
+      uint4 kr[ROWS_PER_GROUP], vr[ROWS_PER_GROUP];
+#pragma unroll
+      for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) {
+        const int row = min(row0 + rr, nrows - 1);
+        kr[rr] = __ldg(reinterpret_cast<const uint4*>(Kc + base + (size_t)row * D + sub * 8));
+      }
+#pragma unroll
+      for (int rr = 0; rr < ROWS_PER_GROUP; ++rr) {
+        const int row = min(row0 + rr, nrows - 1);
+        vr[rr] = __ldg(reinterpret_cast<const uint4*>(Vc + base + (size_t)row * D + sub * 8));
+      }
+      float v[16];
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        float kf[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) kf[i] = bf16_elem(kr[rr], i);
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          F2 acc = f2m(qv[g].v[0], qv[g].v[1], kf[0], kf[1]);
+          acc = f2fma(qv[g].v[2], qv[g].v[3], kf[2], kf[3], acc);
+          acc = f2fma(qv[g].v[4], qv[g].v[5], kf[4], kf[5], acc);
+          acc = f2fma(qv[g].v[6], qv[g].v[7], kf[6], kf[7], acc);
+          v[g * 8 + rr] = f2sum(acc);
+        }
+      }
+#pragma unroll
+      for (int st_ = 0; st_ < 4; ++st_) {
+        const int off = 8 >> st_;
+        const bool upper = (sub & off) != 0;
+#pragma unroll
+        for (int i = 0; i < off; ++i) {
+          const float send = upper ? v[i] : v[i + off];
+          const float keep = upper ? v[i + off] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      }
+      const int gl = sub >> 3, rl = sub & 7;
+      const float s_me = (row0 + rl < nrows) ? v[0] + bias2 : -INFINITY;
+      float mx = s_me;
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      const float m_old = gl ? st[1].m : st[0].m;
+      const float m_new = mx > -INFINITY ? fmaxf(m_old, mx) : m_old;
+      const float pr = mx > -INFINITY ? exp2f(s_me - m_new) : 0.f;
+      float ps = pr;
+      ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+      ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+      ps += __shfl_xor_sync(0xffffffffu, ps, 4);
+      const float m_oth = __shfl_xor_sync(0xffffffffu, m_new, 8);
+      const float ps_oth = __shfl_xor_sync(0xffffffffu, ps, 8);
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        const float mn = (g == gl) ? m_new : m_oth;
+        const float pg = (g == gl) ? ps : ps_oth;
+        const float corr = st[g].m == mn ? 1.f : exp2f(st[g].m - mn);
+        st[g].l = st[g].l * corr + pg;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) st[g].acc[i] *= corr;
+        st[g].m = mn;
+      }
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        float vf[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) vf[i] = bf16_elem(vr[rr], i);
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          const float pg = __shfl_sync(0xffffffffu, pr, g * 8 + rr, 16);
+          f2acc8(st[g].acc, pg, vf);
+        }
+      }
+    } else if constexpr (kRaw) {
       // bf16: the block's key and value rows are all requested before any
       // arithmetic (one memory latency per block), and held as raw 16-byte
       // words, which costs the registers that eight converted rows would
