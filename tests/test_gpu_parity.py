@@ -399,7 +399,7 @@ def test_bwd_sparse_full_budget_matches_training():
         assert rel_err(np64(b), np64(a)) < 1e-2
 
 
-@pytest.mark.parametrize("k", [8, 32])
+@pytest.mark.parametrize("k", [8, 16, 32, 64])
 def test_bwd_sparse_prefill_full_size_one_group(k):
     """Planted prefill workload N=65536, 32/8 heads, sparse K, computed in full
     on the GPU; every gradient of kv-group 0 against the oracle."""
