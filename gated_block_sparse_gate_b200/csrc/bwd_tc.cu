@@ -330,9 +330,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       bulk_wait_group0();  // reductions reach global memory before the CTA exits
       if (*abort_flag) {
         // let loads still in flight land before the CTA exits
-        mbar_wait(&bars->kv_full, 0, abort_flag, nullptr, 1000000ull);
+        mbar_drain(&bars->kv_full, 0, 1000000ull);
         for (int j = issued - kQStages < 0 ? 0 : issued - kQStages; j < issued; ++j)
-          mbar_wait(&bars->q_full[j % kQStages], (j / kQStages) & 1, abort_flag, nullptr, 1000000ull);
+          mbar_drain(&bars->q_full[j % kQStages], (j / kQStages) & 1, 1000000ull);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -410,7 +410,10 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         }
       }
       mma_commit(&bars->done);
-      mbar_wait(&bars->done, 0, abort_flag, a.err, kTimeoutNs);
+      // after an abort the flag cuts the wait short: drain the MMAs still in
+      // flight before tensor memory is freed
+      if (!mbar_wait(&bars->done, 0, abort_flag, a.err, kTimeoutNs))
+        mbar_drain(&bars->done, 0, 1000000ull);
     }
   } else if (warp < kComputeWarps) {
     // ------------------------------------------------------- compute warps

@@ -219,10 +219,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         issued = j + 1;
       }
       if (*abort_flag) {
-        mbar_wait(&bars->q_full, 0, abort_flag, nullptr, 1000000ull);
+        mbar_drain(&bars->q_full, 0, 1000000ull);
         if (issued > 0) {
-          mbar_wait(&bars->k_full, (issued - 1) & 1, abort_flag, nullptr, 1000000ull);
-          mbar_wait(&bars->v_full, (issued - 1) & 1, abort_flag, nullptr, 1000000ull);
+          mbar_drain(&bars->k_full, (issued - 1) & 1, 1000000ull);
+          mbar_drain(&bars->v_full, (issued - 1) & 1, 1000000ull);
         }
       }
     }
@@ -260,7 +260,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
       }
       // drain: every MMA issued above has finished once this arrives
       mma_commit(&bars->drain);
-      mbar_wait(&bars->drain, 0, abort_flag, a.err, kTimeoutNs);
+      // after an abort the flag cuts the wait short: drain the MMAs still in
+      // flight before tensor memory is freed
+      if (!mbar_wait(&bars->drain, 0, abort_flag, a.err, kTimeoutNs))
+        mbar_drain(&bars->drain, 0, 1000000ull);
     }
   } else {
     // ----------------------------------------------------- softmax + epilogue

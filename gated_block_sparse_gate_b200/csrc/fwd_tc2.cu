@@ -175,10 +175,10 @@ fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         issued = j + 1;
       }
       if (*abort_flag) {
-        mbar_wait(&bars->q_full, 0, abort_flag, nullptr, 1000000ull);
+        mbar_drain(&bars->q_full, 0, 1000000ull);
         for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j) {
-          mbar_wait(&bars->k_full[j & 1], (j >> 1) & 1, abort_flag, nullptr, 1000000ull);
-          mbar_wait(&bars->v_full[j & 1], (j >> 1) & 1, abort_flag, nullptr, 1000000ull);
+          mbar_drain(&bars->k_full[j & 1], (j >> 1) & 1, 1000000ull);
+          mbar_drain(&bars->v_full[j & 1], (j >> 1) & 1, 1000000ull);
         }
       }
     }
@@ -228,7 +228,10 @@ fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (ok && j + 1 < n_stages) ok = issue_s(1, j + 1);
       }
       mma_commit(&bars->done);
-      mbar_wait(&bars->done, 0, abort_flag, a.err, kTimeoutNs);
+      // after an abort the flag cuts the wait short: drain the MMAs still in
+      // flight before tensor memory is freed
+      if (!mbar_wait(&bars->done, 0, abort_flag, a.err, kTimeoutNs))
+        mbar_drain(&bars->done, 0, 1000000ull);
     }
   } else {
     // ------------------------------------------------------------- softmax
