@@ -1,30 +1,32 @@
 // fwd_tc2.cu — K2, training mode: gated flash-attention forward with two query
-// tiles per CTA in ping-pong on the tcgen05 tensor cores (sm_100a).
+// tiles per CTA on the tcgen05 tensor cores (sm_100a).
 //
 // Same result as fwd_tc.cu (z_ij = scale q_i.k_j + b_ij with the normalised
 // log gate of the historical key block, 0 with the causal mask on the current
 // block; ai.viyan.live, "SAS Learns Token Importance for Sparse Attention",
 // "The Logit Injection Mechanism"; HF paper page of "SAS: Simple Attention
 // Sparsification via End-to-End Optimization of Context Ranking", Abstract),
-// organised so the tensor cores never wait for one softmax:
+// organised so that the tensor cores never wait for a softmax:
 //
 //  * a CTA owns the same 128-row query tile of two q-heads (A, B) of one kv
 //    group; in training mode both attend exactly the blocks 0..r, so every
 //    K/V stage (two 64-key context blocks) is loaded once for both tiles;
-//  * TMEM: S_A, S_B (128 fp32 columns each), O_A, O_B (128 each); P is written
-//    back as bf16 over the first 64 columns of its S and fed to PV from TMEM;
-//  * the MMA issuer interleaves PV_A(j), S_A(j+1), PV_B(j), S_B(j+1): while
-//    softmax A works on S_A(j+1) the tensor cores run tile B's MMAs and vice
-//    versa;
-//  * softmax warps (one query row per thread) handle each 64-key slot with one
-//    uniform code path (full gate bias, causal current block or masked): the
-//    per-slot raw max comes first, then each logit costs one FFMA with the
-//    slot constant (bias - running max) and one ex2;
-//  * the O rescale is lazy (running max moves only when it grows by > 2^8);
-//    O of a tile is quiescent whenever its next S has landed, because the
-//    commit of that S covers the tile's previous PV.
-// Warps: 0-3 softmax A, 4-7 softmax B, 8 TMA producer, 9 TMEM + MMA issuer.
-// Every mbarrier wait is bounded and reports GBS_ERR_TIMEOUT.
+//  * TMEM: one 128-column S buffer that the two tiles take in turn, P_A and
+//    P_B (64 columns each, bf16 pairs), O_A and O_B (128 each);
+//  * a softmax copies its whole S tile into registers and releases the
+//    buffer at once, so the next tile's S is computed while it works; the
+//    MMA issuer runs S_A(j+1), PV_A(j), S_B(j+1), PV_B(j) and each S only
+//    waits for the other tile's copy of the previous S, never for a P;
+//  * softmax warps (one query row per thread, 208 registers after the
+//    control warpgroup hands its registers over) take each 64-key slot with
+//    one code path (full gate bias, causal current block or masked): the
+//    slot's raw max first, then one FFMA with the slot constant
+//    (bias - running max) and one ex2 per logit;
+//  * the O rescale is lazy (the running max moves only when it grows by more
+//    than 2^8); before it writes P a softmax waits for its tile's previous
+//    PV, which also makes O quiescent for a rescale.
+// Warps: 0-3 softmax A, 4-7 softmax B, 8 TMA producer, 9 TMEM + MMA issuer,
+// 10-11 idle. Every mbarrier wait is bounded and reports GBS_ERR_TIMEOUT.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -40,11 +42,20 @@ using namespace sm100;
 constexpr int kBM = 128;
 constexpr int kSlot = 64;
 constexpr int kBN = 2 * kSlot;
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 constexpr int kTmemCols = 512;
+// registers per thread: 168 at launch (65536 / 384, rounded down to 8); the
+// control warpgroup drops to 72 and the two softmax warpgroups rise to 208:
+// 128 x (208 + 208 + 72) = 62464 <= 384 x 168 = 64512, and per sub-partition
+// (one warp of each warpgroup) 32 x 488 = 15616 <= 16384
+constexpr int kRegsSoftmax = 208;
+constexpr int kRegsControl = 72;
+static_assert(128 * (2 * kRegsSoftmax + kRegsControl) <= kThreads * 168, "register split");
 constexpr uint64_t kTimeoutNs = 4000000000ull;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int kChunk = 128 * 128;  // 64 columns x 128 rows of bf16
+// TMEM columns
+constexpr uint32_t kColS = 0, kColP = 128, kColO = 256;
 
 template <int D>
 struct Layout2 {
@@ -61,7 +72,7 @@ struct Layout2 {
 struct Bars2 {
   uint64_t q_full;
   uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
-  uint64_t s_full[2], p_full[2];
+  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];  // [tile]
   uint64_t done;
   uint32_t tmem_base;
   int abort_flag;
@@ -93,6 +104,14 @@ __device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 template <int D>
@@ -126,7 +145,9 @@ fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
       mbar_init(&bars->s_full[s], 1);
+      mbar_init(&bars->s_free[s], 128);
       mbar_init(&bars->p_full[s], 128);
+      mbar_init(&bars->pv_done[s], 1);
     }
     mbar_init(&bars->done, 1);
     bars->abort_flag = 0;
@@ -142,8 +163,10 @@ fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort_flag = &bars->abort_flag;
 
-  if (warp == 8) {
-    if (lane == 0) {
+  if (warp >= 8) {
+    regs_dec<kRegsControl>();
+    if (warp == 8 && lane == 0) {
+      // ---------------------------------------------------------- TMA producer
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
@@ -175,36 +198,42 @@ fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         issued = j + 1;
       }
       if (*abort_flag) {
+        // let loads still in flight land before the CTA exits
         mbar_drain(&bars->q_full, 0, 1000000ull);
         for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j) {
           mbar_drain(&bars->k_full[j & 1], (j >> 1) & 1, 1000000ull);
           mbar_drain(&bars->v_full[j & 1], (j >> 1) & 1, 1000000ull);
         }
       }
-    }
-  } else if (warp == 9) {
-    if (lane == 0) {
+    } else if (warp == 9 && lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
       constexpr uint32_t idS = idesc_bf16_f32(kBM, kBN, 0);
       constexpr uint32_t idO = idesc_bf16_f32(kBM, D, 1);
       const uint32_t qa = smem_u32(smem + L::kQAOff), qb = smem_u32(smem + L::kQBOff);
+      // S_x(j) = Q_x K_j^T into the shared S buffer
       auto issue_s = [&](int x, int j) -> bool {
         const int st = j & 1;
         if (x == 0) {
           if (!mbar_wait(&bars->k_full[st], (j >> 1) & 1, abort_flag, a.err, kTimeoutNs)) return false;
-          tc_fence_after();
         }
+        // the buffer is free once the other tile has copied its previous S out
+        if (!(x == 0 && j == 0) &&
+            !mbar_wait(&bars->s_free[x ^ 1], (x ? j : j - 1) & 1, abort_flag, a.err, kTimeoutNs))
+          return false;
+        tc_fence_after();
         const uint32_t q_addr = x ? qb : qa;
         const uint32_t k_addr = smem_u32(smem + L::kKOff + st * L::kTile);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const int ch = ks >> 2, kk = ks & 3;
-          mma_ss(tmem + x * 128, sdesc_sw128(q_addr + ch * kChunk + kk * 32, 16, 1024),
+          mma_ss(tmem + kColS, sdesc_sw128(q_addr + ch * kChunk + kk * 32, 16, 1024),
                  sdesc_sw128(k_addr + ch * kChunk + kk * 32, 16, 1024), idS, ks > 0 ? 1u : 0u);
         }
         mma_commit(&bars->s_full[x]);
         if (x == 1) mma_commit(&bars->k_empty[st]);
         return true;
       };
+      // O_x += P_x(j) V_j, P from its own TMEM columns
       auto issue_pv = [&](int x, int j) -> bool {
         const int st = j & 1;
         if (!mbar_wait(&bars->p_full[x], j & 1, abort_flag, a.err, kTimeoutNs)) return false;
@@ -214,18 +243,19 @@ fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const uint32_t v_addr = smem_u32(smem + L::kVOff + st * L::kTile);
 #pragma unroll
         for (int ks = 0; ks < kBN / 16; ++ks)
-          mma_ts(tmem + 256 + x * 128, tmem + x * 128 + ks * 8,
+          mma_ts(tmem + kColO + x * 128, tmem + kColP + x * 64 + ks * 8,
                  sdesc_sw128(v_addr + ks * 2048, kChunk, 1024), idO, (j > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(&bars->pv_done[x]);
         if (x == 1) mma_commit(&bars->v_empty[st]);
         return true;
       };
       bool ok = mbar_wait(&bars->q_full, 0, abort_flag, a.err, kTimeoutNs);
       ok = ok && issue_s(0, 0) && issue_s(1, 0);
       for (int j = 0; ok && j < n_stages; ++j) {
-        ok = issue_pv(0, j);
-        if (ok && j + 1 < n_stages) ok = issue_s(0, j + 1);
-        if (ok) ok = issue_pv(1, j);
+        if (j + 1 < n_stages) ok = issue_s(0, j + 1);
+        if (ok) ok = issue_pv(0, j);
         if (ok && j + 1 < n_stages) ok = issue_s(1, j + 1);
+        if (ok) ok = issue_pv(1, j);
       }
       mma_commit(&bars->done);
       // after an abort the flag cuts the wait short: drain the MMAs still in
@@ -234,14 +264,15 @@ fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         mbar_drain(&bars->done, 0, 1000000ull);
     }
   } else {
+    regs_inc<kRegsSoftmax>();
     // ------------------------------------------------------------- softmax
     const int x = warp >> 2, quad = warp & 3;
     const int row = quad * 32 + lane;
     const int half = row >> 6, iloc = row & 63;
     const int myr = 2 * tile + half;
     const int bh = x ? bhB : bhA;
-    const uint32_t tS = tmem + ((uint32_t)(quad * 32) << 16) + x * 128;
-    const uint32_t tO = tS + 256;
+    const uint32_t tLane = tmem + ((uint32_t)(quad * 32) << 16);
+    const uint32_t tS = tLane + kColS, tP = tLane + kColP + x * 64, tO = tLane + kColO + x * 128;
     const float sc = p.scale_log2;
     const size_t srow = (size_t)bh * p.Nb + myr;
     float m = -INFINITY, l = 0.f;
@@ -268,82 +299,75 @@ fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         break;
       }
       tc_fence_after();
-      // pass 1: per-slot maximum of the scaled, biased logits; slot 1 stays in
-      // registers, slot 0 is read again in pass 2 (keeps register use low)
-      uint32_t v1[64];
+      // copy the whole S tile out and hand the buffer to the other tile
+      uint32_t v[128];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(v + q * 32));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bars->s_free[x]);
       float smax[2];
 #pragma unroll
       for (int s = 0; s < 2; ++s) {
-        uint32_t v[64];
-        tmem_ld32(tS + s * 64, *reinterpret_cast<uint32_t(*)[32]>(v));
-        tmem_ld32(tS + s * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-        tmem_wait_ld();
+        uint32_t* w = v + s * 64;
         if (kind[s] == kDiag) {
 #pragma unroll
           for (int k = 0; k < 64; ++k)
-            if (k > iloc) v[k] = __float_as_uint(-INFINITY);
+            if (k > iloc) w[k] = __float_as_uint(-INFINITY);
         }
         float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
         for (int k = 0; k < 64; k += 8) {
-          a0 = max3(a0, __uint_as_float(v[k]), __uint_as_float(v[k + 1]));
-          a1 = max3(a1, __uint_as_float(v[k + 2]), __uint_as_float(v[k + 3]));
-          a2 = max3(a2, __uint_as_float(v[k + 4]), __uint_as_float(v[k + 5]));
-          a3 = max3(a3, __uint_as_float(v[k + 6]), __uint_as_float(v[k + 7]));
+          a0 = max3(a0, __uint_as_float(w[k]), __uint_as_float(w[k + 1]));
+          a1 = max3(a1, __uint_as_float(w[k + 2]), __uint_as_float(w[k + 3]));
+          a2 = max3(a2, __uint_as_float(w[k + 4]), __uint_as_float(w[k + 5]));
+          a3 = max3(a3, __uint_as_float(w[k + 6]), __uint_as_float(w[k + 7]));
         }
         const float raw = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
         smax[s] = kind[s] == kMasked ? -INFINITY : fmaf(raw, sc, bias[s]);
-        if (s == 1) {
-#pragma unroll
-          for (int k = 0; k < 64; ++k) v1[k] = v[k];
-        }
       }
       const float mx = fmaxf(smax[0], smax[1]);
       const bool need = mx > m + kRescaleThreshold;
-      if (__any_sync(0xffffffffu, need) && j > 0) {
-        // O is quiescent: the commit that signalled this S covered the previous PV
-        const float f = need ? ex2(m - mx) : 1.f;
-#pragma unroll
-        for (int q = 0; q < D / 32; ++q) {
-          uint32_t o[32];
-          tmem_ld32(tO + q * 32, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
-          tmem_st32(tO + q * 32, o);
+      if (j > 0) {
+        // PV_x(j-1) has read P_x and written O
+        if (!mbar_wait(&bars->pv_done[x], (j - 1) & 1, abort_flag, a.err, kTimeoutNs)) {
+          ok = false;
+          break;
         }
-        if (need) l *= f;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, need)) {
+          const float f = need ? ex2(m - mx) : 1.f;
+#pragma unroll
+          for (int q = 0; q < D / 32; ++q) {
+            uint32_t o[32];
+            tmem_ld32(tO + q * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
+            tmem_st32(tO + q * 32, o);
+          }
+          if (need) l *= f;
+        }
       }
       if (need) m = mx;
       const float mu = m == -INFINITY ? 0.f : m;
       float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
-      // pass 2, slot 0: 32-column chunks; bf16 P of keys [32c, 32c+32) goes to
-      // columns [16c, 16c+16), which this pass has already read
+      // P of keys [32c, 32c + 32) -> P_x columns [16c, 16c + 16)
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < 4; ++c) {
+        const int s = c >> 1;
         uint32_t pk[16];
-        if (kind[0] == kMasked) {
+        if (kind[s] == kMasked) {
 #pragma unroll
           for (int k = 0; k < 16; ++k) pk[k] = 0u;
         } else {
-          uint32_t v[32];
-          tmem_ld32(tS + c * 32, v);
-          tmem_wait_ld();
-          const float cst = bias[0] - mu;
+          const float cst = bias[s] - mu;
 #pragma unroll
           for (int k = 0; k < 32; k += 4) {
-            float x0 = fmaf(__uint_as_float(v[k]), sc, cst);
-            float x1 = fmaf(__uint_as_float(v[k + 1]), sc, cst);
-            float x2 = fmaf(__uint_as_float(v[k + 2]), sc, cst);
-            float x3 = fmaf(__uint_as_float(v[k + 3]), sc, cst);
-            if (kind[0] == kDiag) {
-              const int kk = c * 32 + k;
-              if (kk > iloc) x0 = -INFINITY;
-              if (kk + 1 > iloc) x1 = -INFINITY;
-              if (kk + 2 > iloc) x2 = -INFINITY;
-              if (kk + 3 > iloc) x3 = -INFINITY;
-            }
-            const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+            const float p0 = ex2(fmaf(__uint_as_float(v[c * 32 + k]), sc, cst));
+            const float p1 = ex2(fmaf(__uint_as_float(v[c * 32 + k + 1]), sc, cst));
+            const float p2 = ex2(fmaf(__uint_as_float(v[c * 32 + k + 2]), sc, cst));
+            const float p3 = ex2(fmaf(__uint_as_float(v[c * 32 + k + 3]), sc, cst));
             l0 += p0;
             l1 += p1;
             l2 += p2;
@@ -352,31 +376,7 @@ fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             pk[k / 2 + 1] = cvt_bf16x2(p2, p3);
           }
         }
-        tmem_st16(tS + c * 16, pk);
-      }
-      // slot 1 from registers -> columns [32, 64) (slot 0's upper half, read above)
-      {
-        uint32_t pk[32];
-        if (kind[1] == kMasked) {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) pk[k] = 0u;
-        } else {
-          const float cst = bias[1] - mu;
-#pragma unroll
-          for (int k = 0; k < 64; k += 4) {
-            const float p0 = ex2(fmaf(__uint_as_float(v1[k]), sc, cst));
-            const float p1 = ex2(fmaf(__uint_as_float(v1[k + 1]), sc, cst));
-            const float p2 = ex2(fmaf(__uint_as_float(v1[k + 2]), sc, cst));
-            const float p3 = ex2(fmaf(__uint_as_float(v1[k + 3]), sc, cst));
-            l0 += p0;
-            l1 += p1;
-            l2 += p2;
-            l3 += p3;
-            pk[k / 2] = cvt_bf16x2(p0, p1);
-            pk[k / 2 + 1] = cvt_bf16x2(p2, p3);
-          }
-        }
-        tmem_st32(tS + 32, pk);
+        tmem_st16(tP + c * 16, pk);
       }
       l += (l0 + l1) + (l2 + l3);
       tmem_wait_st();
