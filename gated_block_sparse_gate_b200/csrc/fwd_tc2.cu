@@ -448,8 +448,14 @@ cudaError_t launch2(const Fwd2Args& a, const void* Q, const void* K, const void*
       !make_map2(&tv, V, D, p.N, p.B * p.Hkv, kSlot))
     return cudaErrorInvalidValue;
   auto kern = fwd_tc2_kernel<D>;
+  // setmaxnreg.inc waits until the registers it asks for are free: launch only
+  // if the kernel starts with enough registers per thread for the split
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs * kThreads < 128 * (2 * kRegsSoftmax + kRegsControl)) return cudaErrorInvalidConfiguration;
   const int smem = Layout2<D>::kSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)(p.B * (p.Hq / 2) * a.n_tiles);
   timer_begin(GBS_OP_FWD, st);
