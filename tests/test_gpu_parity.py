@@ -510,7 +510,10 @@ def test_run_to_run_determinism():
     In the backward dK and dV accumulate inside one CTA (bitwise too); dQ and the
     tile sums behind dS are summed across CTAs in hardware order, so they repeat
     to within fp32 rounding: dS (fp32) to 1e-5, and dQ, that fp32 sum rounded
-    once to bf16, to within one bf16 ulp of each element."""
+    once to bf16, to within one bf16 ulp of each element plus the fp32 rounding
+    of the sum itself, which an element that cancels can expose (2^-16 of the
+    largest |dQ| here: 16 key tiles, each change of order worth a few fp32 ulps
+    of the partial sums)."""
     x = _dev(_small(61, 1, 8, 2, 1024, 128, torch.bfloat16, scaled=False))
     for mode, k in (("train", 0), ("sparse", 3)):
         O1, L1 = gb.forward(x["Q"], x["K"], x["V"], x["S"], mode=mode, topk=k)
@@ -520,7 +523,8 @@ def test_run_to_run_determinism():
         g2 = gb.backward(x["Q"], x["K"], x["V"], x["S"], O1, L1, x["dO"], mode=mode, topk=k)
         assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2]), mode
         a, b = np64(g1[0]), np64(g2[0])
-        assert np.all(np.abs(a - b) <= 2.0 ** -8 * np.maximum(np.abs(a), np.abs(b)) + 1e-30), mode
+        floor = 2.0 ** -16 * max(np.abs(a).max(), np.abs(b).max())
+        assert np.all(np.abs(a - b) <= 2.0 ** -8 * np.maximum(np.abs(a), np.abs(b)) + floor), mode
         assert rel_err(np64(g1[3]), np64(g2[3])) < 1e-5, mode
     from dataclasses import replace
     w = replace(WORKLOADS["sparse_decode_bf16_b64_l131072"], B=4, N=5000)
